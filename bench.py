@@ -1,0 +1,482 @@
+"""Benchmark of the streaming KV-cache attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload ID]
+
+A step is one window step of the whole hot path over every layer of the
+workload: for each layer, kv_stream_insert of the new frame of each view plus
+the text (evicting each view's oldest frame), then stream_attn of the step's
+queries against the layer's cache. Default workload: the driving-shaped window
+(4 cameras x 4 frames x 180 tokens + 256 text tokens, 36 layers, H=32, Hkv=8,
+d=128), synthetic seeded inputs resident in HBM before timing.
+
+Prints ONE JSON line (rank 0). ``value`` is algorithmic attention TFLOP/s of the
+whole job (4*d*H per visible query-key pair, summed over layers and ranks),
+timed on the device with CUDA events between two barriers, max over ranks.
+Under torchrun each rank runs its own replica of the workload (weak scaling,
+no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "stream-attn TFLOP/s & µs/window-step (4 cams×4 frames); % of B200 BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0
+KERNEL_SOURCES = ["streaming_kv_cache_stream_b200/csrc/stream_attn.cu",
+                  "streaming_kv_cache_stream_b200/csrc/sm100.cuh",
+                  "streaming_kv_cache_stream_b200/csrc/fs_internal.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "stream_attn_traffic.txt")
+
+
+# ------------------------------------------------------------------ helpers
+
+def visible_pairs_step(V, T, n, X):
+    """Visible (query, key) pairs of one window step: view v's new-frame token i
+    sees v*T*n + (T-1)*n + i + 1 keys, text token j sees V*T*n + j + 1."""
+    frames = V * n * ((T - 1) * n + 1) + T * n * n * V * (V - 1) // 2 + V * n * (n - 1) // 2
+    text = X * (V * T * n + 1) + X * (X - 1) // 2
+    return frames + text
+
+
+def step_flops(wl):
+    return 4.0 * wl.d * wl.H * visible_pairs_step(wl.views, wl.frames, wl.tok_per_frame, wl.text_len)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_id):
+    """DRAM bytes per stream_attn launch from a committed ncu summary, if it was
+    taken on the current kernel source and this workload; else None."""
+    try:
+        kv = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("kernel_sha256_16") != kernel_hash() or kv.get("workload_id") != str(workload_id):
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["no samples"]}
+        load = sorted(sm)[len(sm) // 4:] or sm  # drop the idle lead-in samples
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_id(dev):
+    """nvidia-smi id of a torch device: its UUID when torch exposes it."""
+    import torch
+
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index or 0)
+
+
+def dist_setup(n_gpus):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------- CPU oracle leg
+
+def oracle_timing(wid, target_s=15.0, max_units=64):
+    """Times the fp64 CPU oracle (as it stands) on window steps of this workload.
+
+    Returns (seconds, algorithmic flops, layer-steps done, threads used)."""
+    import numpy as np
+
+    from oracle import StreamOracle, bf16_bits_to_f64
+    from streaming_kv_cache_stream_b200.inputs import WORKLOADS, window_inputs
+
+    wl = WORKLOADS[wid]
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    fl = step_flops(wl)
+    total_s, units, layer = 0.0, 0, 0
+    while units < max_units and total_s < target_s:
+        orc = StreamOracle(wl.views, wl.frames, wl.tok_per_frame, wl.text_len, wl.H, wl.Hkv, wl.d, wl.rope_base)
+        pre = window_inputs(wid, layer % wl.layers, 0)
+        orc.win.prefill(bf16_bits_to_f64(pre["K"]), bf16_bits_to_f64(pre["V"]))  # untimed setup
+        inp = window_inputs(wid, layer % wl.layers, 1)
+        f = {x: bf16_bits_to_f64(inp[x]) for x in ("Q", "K", "V")}
+        t0 = time.perf_counter()
+        orc.step(f["Q"], f["K"], f["V"])
+        total_s += time.perf_counter() - t0
+        units += 1
+        layer += 1
+    return total_s, fl * units, units, threads
+
+
+# --------------------------------------------------------------- GPU leg
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    from streaming_kv_cache_stream_b200.abi import Stream, load
+    from streaming_kv_cache_stream_b200.inputs import WORKLOADS, window_inputs
+
+    world, rank, local = dist_setup(args.gpus)
+    load()
+    wid = args.workload
+    wl = WORKLOADS[wid]
+    layers = wl.layers
+    dev = torch.device("cuda", local if world > 1 else 0)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    streams = [Stream(wl.views, wl.frames, wl.tok_per_frame, wl.text_len, wl.H, wl.Hkv, wl.d, wl.rope_base)
+               for _ in range(layers)]
+    # prefill (the stream's first call), untimed
+    for l, s in enumerate(streams):
+        inp = window_inputs(wid, l, 0)
+        q = to_dev(inp["Q"])
+        out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        s.insert(to_dev(inp["K"]), to_dev(inp["V"]))
+        s.attend(q, out)
+        del q, out
+    torch.cuda.synchronize()
+    # step inputs resident in HBM: `sets` distinct input sets per layer, cycled
+    sets = 2
+    inputs = [[{x: to_dev(window_inputs(wid, l, 1 + k)[x]) for x in ("Q", "K", "V")} for k in range(sets)]
+              for l in range(layers)]
+    nq = wl.step_tokens
+    outs = [torch.empty((nq, wl.H, wl.d), dtype=torch.float32, device=dev) for _ in range(layers)]
+    stream = torch.cuda.current_stream()
+
+    def step(k, ev=None):
+        for l, s in enumerate(streams):
+            inp = inputs[l][k % sets]
+            if ev is not None:
+                ev[l][0].record(stream)
+            s.insert(inp["K"], inp["V"])
+            if ev is not None:
+                ev[l][1].record(stream)
+            s.attend(inp["Q"], outs[l])
+            if ev is not None:
+                ev[l][2].record(stream)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    launches0 = sum(s.info().launches for s in streams)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(layers)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(gpu_id(dev)) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            step(args.warmup + k, evs[k])
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    launches = sum(s.info().launches for s in streams) - launches0
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
+    ins_ms = [evs[k][l][0].elapsed_time(evs[k][l][1]) for k in range(args.steps) for l in range(layers)]
+    att_ms = [evs[k][l][1].elapsed_time(evs[k][l][2]) for k in range(args.steps) for l in range(layers)]
+
+    fl_layer = step_flops(wl)
+    ms_per_step = elapsed_ms / args.steps
+    value = world * fl_layer * layers / (ms_per_step * 1e-3) / 1e12
+    att_avg_ms = statistics.mean(att_ms)
+    att_tflops = fl_layer / (att_avg_ms * 1e-3) / 1e12
+    ins_bytes = 4.0 * wl.step_tokens * wl.Hkv * wl.d * 2  # read K_new, V_new + write both into the ring
+    ins_avg_ms = statistics.mean(ins_ms)
+    peaks, src = load_peaks()
+    peak_t = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    hbm = float(peaks.get("hbm_gbs"))
+
+    # ---- end to end through the public C ABI with host buffers
+    e2e_steps = max(1, min(args.steps, 5))
+    pin = [{x: torch.from_numpy(np.ascontiguousarray(window_inputs(wid, l, 1)[x]).view(np.int16)).pin_memory()
+            for x in ("Q", "K", "V")} for l in range(layers)]
+    pin_out = [torch.empty((nq, wl.H, wl.d), dtype=torch.float32).pin_memory() for _ in range(layers)]
+    for l, s in enumerate(streams):  # first call sizes the staging buffers, untimed
+        s.step_host(pin[l]["K"], pin[l]["V"], pin[l]["Q"], pin_out[l])
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(e2e_steps):
+        for l, s in enumerate(streams):
+            s.step_host(pin[l]["K"], pin[l]["V"], pin[l]["Q"], pin_out[l])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = layers * (2 * wl.step_tokens * wl.Hkv * wl.d * 2 + nq * wl.H * wl.d * 2)
+    d2h = layers * nq * wl.H * wl.d * 4
+
+    result = None
+    if rank == 0:
+        traffic = recorded_traffic(wid)
+        result = {
+            "metric": METRIC,
+            "value": round(value, 3),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 5),
+            "us_per_window_step": round(ms_per_step * 1e3, 2),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f16",
+            "precision": "bf16 inputs; rotated Q/K as fp16 hi+lo (3 MMAs), P and V fp16, fp32 accumulate, fp32 out",
+            "data": "synthetic",
+            "config": {
+                "workload": f"{wl.name} window: {wl.views} cams x {wl.frames} frames x {wl.tok_per_frame} tok "
+                            f"+ {wl.text_len} text, {wl.layers} layers, H{wl.H}/Hkv{wl.Hkv}/d{wl.d}",
+                "workload_id": wid,
+                "layers": layers,
+                "window_len": wl.window_len,
+                "queries_per_step": nq,
+                "algorithmic_gflop_per_layer_step": round(fl_layer / 1e9, 4),
+                "l2": "inputs larger than L2: each step streams ~%.2f GB of per-layer inputs, caches and outputs"
+                      % (layers * (wl.step_tokens * (2 * wl.Hkv + wl.H) * wl.d * 2 + nq * wl.H * wl.d * 4
+                                   + 2 * wl.window_len * wl.Hkv * wl.d * 2) / 1e9),
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            },
+            "roofline": {
+                "bound": "tensor",
+                "kernel": "stream_attn",
+                "achieved": round(att_tflops, 2),
+                "peak": peak_t,
+                "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
+                "unit": "TFLOP/s",
+                "frac": round(att_tflops / peak_t, 4),
+                "frac_of_nominal_2250": round(att_tflops / NOMINAL_BF16_TFLOPS, 4),
+                "traffic": traffic,
+                "us_per_launch": round(att_avg_ms * 1e3, 2),
+            },
+            "insert": {
+                "kernel": "kv_stream_insert",
+                "bound": "hbm",
+                "us_per_launch": round(ins_avg_ms * 1e3, 2),
+                "bytes_per_launch": ins_bytes,
+                "achieved_gbs": round(ins_bytes / (ins_avg_ms * 1e-3) / 1e9, 1),
+                "peak_gbs": hbm,
+                "frac": round(ins_bytes / (ins_avg_ms * 1e-3) / 1e9 / hbm, 4),
+            },
+            "e2e": {
+                "value": round(world * fl_layer * layers / (e2e_ms * 1e-3) / 1e12, 3),
+                "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "api": "fs_stream_step_host, pinned host buffers",
+            },
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+    for s in streams:
+        s.close()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_reference(args):
+    """The oracle arm: the fp64 CPU oracle, as it stands, on host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    from streaming_kv_cache_stream_b200.inputs import WORKLOADS
+
+    wid = args.workload
+    wl = WORKLOADS[wid]
+    times = []
+    flops = 0.0
+    threads = 1
+    units_total = 0
+    for _ in range(args.warmup):
+        oracle_timing(wid, target_s=0.0, max_units=1)
+    for _ in range(args.steps):
+        s, fl, units, threads = oracle_timing(wid, target_s=8.0, max_units=36)
+        times.append(s)
+        flops += fl
+        units_total += units
+    total = sum(times)
+    value = flops / total / 1e12
+    per_layer_ms = total / units_total * 1e3
+    sample = (f"{units_total} layer-steps of the workload (one window step of one layer each: "
+              f"{wl.step_tokens} queries x {wl.window_len} keys, all {wl.H} heads), fp64 numpy")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": per_layer_ms * wl.layers,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name} window, {wl.layers} layers", "workload_id": wid,
+                   "note": "ms_per_step scales the per-layer time by the layer count"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        res = run_reference(args)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    res = run_ours(args)
+    if res is not None:
+        if res["n_gpus"] == 1 and not args.no_cpu_baseline:
+            s, fl, units, threads = oracle_timing(args.workload)
+            from streaming_kv_cache_stream_b200.inputs import WORKLOADS
+
+            wl = WORKLOADS[args.workload]
+            res["cpu_baseline"] = {
+                "value": round(fl / s / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                "sample": f"{units} layer-steps ({wl.step_tokens} queries x {wl.window_len} keys, {wl.H} heads each), "
+                          f"{s:.1f} s of fp64 numpy",
+            }
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,103 @@
+// fs_internal.cuh -- parameters shared by the host side of the library and its
+// kernels, and the position arithmetic of the view-major window.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fs {
+
+constexpr int kTileRows = 128;          // query rows (token x head) and keys per tile
+constexpr int kMaxKeyTiles = 2048;      // key rows per kv head <= 2048 * 128
+constexpr int kMaxVerify = 256;         // scratch rows for a drafted block (FS_MAX_VERIFY_TOKENS)
+constexpr unsigned kErrTimeout = 1u;    // device error word bits
+constexpr unsigned kErrBadLaunch = 2u;
+
+enum QueryMode : int { kQueryPrefill = 0, kQueryStep = 1, kQueryVerify = 2 };
+
+// Shape of the view-major window and the ring head, as the kernels need them.
+struct WindowShape {
+    int V, T, n, X;     // views, frames per view, tokens per frame, text tokens
+    int ring_rows;      // V * T * n
+    int head;           // ring slot holding every view's oldest frame
+};
+
+// Window position of physical cache row `row` (per kv head).
+// Ring rows: view v, slot s, token i sit at row (v*T + s)*n + i; the slot's
+// age in the window is (s - head) mod T (0 = oldest), so the token's position
+// in the current view-major window is v*T*n + age*n + i. Text rows (and the
+// drafted block after them) keep their row index as position: they follow all
+// views. "Keys are stored pre-RoPE and rotated at shifted positions"
+// (FlashDrive technical summary, Methodology 1, "Positional Encoding").
+__host__ __device__ __forceinline__ int key_pos(const WindowShape& w, int row) {
+    if (row >= w.ring_rows) return row;
+    const int tn = w.T * w.n;
+    const int v = row / tn;
+    const int rem = row - v * tn;
+    const int s = rem / w.n;
+    const int i = rem - s * w.n;
+    int age = s - w.head;
+    if (age < 0) age += w.T;
+    return v * tn + age * w.n + i;
+}
+
+// Window position of query token t.
+//   prefill: the whole window in order, position t;
+//   step: view v's newest frame (the last of its T frames) then the text,
+//         "inserted at the end of each view's sequence" (FlashDrive technical
+//         summary, Methodology 1, "Token Layout");
+//   verify: a drafted block right after the text.
+__host__ __device__ __forceinline__ int query_pos(const WindowShape& w, int mode, int t) {
+    if (mode == kQueryPrefill) return t;
+    if (mode == kQueryVerify) return w.ring_rows + w.X + t;
+    const int vn = w.V * w.n;
+    if (t < vn) {
+        const int v = t / w.n;
+        const int i = t - v * w.n;
+        return v * w.T * w.n + (w.T - 1) * w.n + i;
+    }
+    return w.ring_rows + (t - vn);
+}
+
+struct AttnParams {
+    WindowShape w;
+    int key_rows;         // valid key rows per kv head for this launch
+    int Hkv, G, H, d;     // kv heads, query heads per kv head, query heads, head dim
+    int nq;               // query tokens
+    int q_mode;           // QueryMode
+    int q_tiles;          // ceil(nq * G / 128)
+    int splits;           // key splits per (kv head, query tile)
+    float q_scale;        // log2(e) / sqrt(d), folded into the rotated queries
+    const float2* rope;   // [rope_rows][d/2] (cos, sin) of pos * theta_i
+    int rope_rows;
+    float* out;           // [nq][H][d] fp32
+    float* part_o;        // [items][splits][128][d] fp32 (splits > 1)
+    float2* part_ml;      // [items][splits][128] (running max in log2 units, sum)
+    unsigned* err;        // device error word
+    unsigned long long wait_limit_ns;
+};
+
+struct InsertParams {
+    const uint4* K_src;   // [N][Hkv][d] bf16 as 16-byte chunks
+    const uint4* V_src;
+    uint4* K_cache;       // [Hkv][rows_cap][d]
+    uint4* V_cache;
+    int N;                // tokens to insert
+    int Hkv;
+    int chunks;           // d * 2 / 16 chunks per (token, kv head) vector
+    int rows_cap;         // rows per kv head in the cache
+    int mode;             // 0: prefill (row = t), 1: step, 2: drafted block (row = L + t)
+    int V, T, n, X, ring_rows, head;
+};
+
+// Launchers (defined in the .cu files); all enqueue on `stream` and return the
+// launch's cudaError_t.
+cudaError_t launch_kv_stream_insert(const InsertParams& p, int num_sms, cudaStream_t stream);
+cudaError_t launch_stream_attn(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tk,
+                               const CUtensorMap& tv, cudaStream_t stream);
+cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_positions(const WindowShape& w, int rows, int* pos_out, cudaStream_t stream);
+cudaError_t launch_wait_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);
+size_t stream_attn_smem_bytes(int d);
+
+}  // namespace fs

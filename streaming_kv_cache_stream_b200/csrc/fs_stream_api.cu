@@ -1,0 +1,472 @@
+// fs_stream_api.cu -- host side of the C ABI declared in include/fs_stream.h:
+// argument checks, the stream state machine (prefill first, then window
+// steps; FlashDrive README, "Library": the first call of a stream only
+// prefills), device allocation of the static cache, TMA tensor maps, and
+// kernel launches. No compute happens on the host: every step of the path runs
+// in the kernels of kv_stream_insert.cu and stream_attn.cu.
+// Tensor maps are built once per handle (for the cache); queries are read by
+// the kernel with plain loads, so attend encodes nothing per call.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include <cudaTypedefs.h>
+
+#include "../../include/fs_stream.h"
+#include "fs_internal.cuh"
+
+using fs::AttnParams;
+using fs::InsertParams;
+using fs::WindowShape;
+
+struct fs_stream {
+    int V, T, n, X, H, Hkv, G, d;
+    float base;
+    int L, ring_rows, step_tokens, rows_cap, rope_rows;
+    int state = FS_STATE_EXPECT_PREFILL;
+    int head = 0;
+    long long steps = 0;
+    int last_insert_tokens = 0;
+    std::vector<long long> slot_frame;  // frame id held by each ring slot (same for all views)
+    cudaStream_t stream = nullptr;
+    int device = 0, num_sms = 148;
+    uint16_t* K_cache = nullptr;
+    uint16_t* V_cache = nullptr;
+    float2* rope = nullptr;
+    unsigned* err = nullptr;
+    float* part_o = nullptr;
+    float2* part_ml = nullptr;
+    int part_rows_cap = 0;  // rows of 128 query rows x d fp32 the split scratch holds
+    void* stage = nullptr;  // host-path staging: K, V, Q, out
+    size_t stage_bytes = 0;
+    CUtensorMap tmap_k, tmap_v;
+    unsigned long long wait_limit_ns = 2000000000ull;
+    long long cache_bytes = 0;
+    long long launches = 0;
+    std::string last_error;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(fs_stream_t s, int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    if (s) s->last_error = buf;
+    return code;
+}
+
+#define FS_CUDA(s, call)                                                                       \
+    do {                                                                                       \
+        cudaError_t e_ = (call);                                                               \
+        if (e_ != cudaSuccess)                                                                 \
+            return fail((s), FS_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));     \
+    } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 3-D bf16 tensor map, 128-byte swizzle, box {64, b1, b2}, out-of-range reads as zero.
+int make_map(fs_stream_t s, CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+             uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b1, uint32_t b2) {
+    auto enc = get_encode();
+    if (!enc) return fail(s, FS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    cuuint32_t box[3] = {64, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(s, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+    return FS_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+WindowShape shape_of(const fs_stream* s) {
+    WindowShape w;
+    w.V = s->V;
+    w.T = s->T;
+    w.n = s->n;
+    w.X = s->X;
+    w.ring_rows = s->ring_rows;
+    w.head = s->head;
+    return w;
+}
+
+void free_all(fs_stream* s) {
+    cudaFree(s->K_cache);
+    cudaFree(s->V_cache);
+    cudaFree(s->rope);
+    cudaFree(s->err);
+    cudaFree(s->part_o);
+    cudaFree(s->part_ml);
+    cudaFree(s->stage);
+}
+
+int check_err_word(fs_stream_t s) {
+    unsigned h = 0;
+    FS_CUDA(s, cudaMemcpy(&h, s->err, sizeof h, cudaMemcpyDeviceToHost));
+    if (h) {
+        FS_CUDA(s, cudaMemset(s->err, 0, sizeof(unsigned)));
+        if (h & fs::kErrTimeout) return fail(s, FS_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up");
+        return fail(s, FS_ERR_CUDA, "device error word 0x%x", h);
+    }
+    return FS_OK;
+}
+
+int do_insert(fs_stream_t s, const void* K, const void* V, int n_tokens, int mode) {
+    InsertParams p;
+    p.K_src = static_cast<const uint4*>(K);
+    p.V_src = static_cast<const uint4*>(V);
+    p.K_cache = reinterpret_cast<uint4*>(s->K_cache);
+    p.V_cache = reinterpret_cast<uint4*>(s->V_cache);
+    p.N = n_tokens;
+    p.Hkv = s->Hkv;
+    p.chunks = s->d * 2 / 16;
+    p.rows_cap = s->rows_cap;
+    p.mode = mode;
+    p.V = s->V;
+    p.T = s->T;
+    p.n = s->n;
+    p.X = s->X;
+    p.ring_rows = s->ring_rows;
+    p.head = s->head;
+    FS_CUDA(s, fs::launch_kv_stream_insert(p, s->num_sms, s->stream));
+    s->launches += 1;
+    return FS_OK;
+}
+
+// Splits of the key range per (kv head, query tile) so that small query sets
+// still fill the SMs; capped by the scratch and by the number of key tiles.
+int choose_splits(const fs_stream* s, int items, int key_rows) {
+    if (items >= s->num_sms) return 1;
+    const int ktiles = (key_rows + fs::kTileRows - 1) / fs::kTileRows;
+    int sp = (s->num_sms + items - 1) / items;
+    if (sp > ktiles / 2) sp = ktiles / 2;
+    if (sp > s->part_rows_cap / items) sp = s->part_rows_cap / items;
+    return sp < 1 ? 1 : sp;
+}
+
+int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key_rows) {
+    const int q_tiles = (nq * s->G + fs::kTileRows - 1) / fs::kTileRows;
+    AttnParams p;
+    p.w = shape_of(s);
+    p.key_rows = key_rows;
+    p.Hkv = s->Hkv;
+    p.G = s->G;
+    p.H = s->H;
+    p.d = s->d;
+    p.nq = nq;
+    p.q_mode = mode;
+    p.q_tiles = q_tiles;
+    p.splits = choose_splits(s, s->Hkv * q_tiles, key_rows);
+    p.q_scale = float(1.4426950408889634 / std::sqrt(double(s->d)));
+    p.rope = s->rope;
+    p.rope_rows = s->rope_rows;
+    p.out = static_cast<float*>(out);
+    p.part_o = s->part_o;
+    p.part_ml = s->part_ml;
+    p.err = s->err;
+    p.wait_limit_ns = s->wait_limit_ns;
+    FS_CUDA(s, fs::launch_stream_attn(p, static_cast<const uint16_t*>(Q), s->tmap_k, s->tmap_v, s->stream));
+    s->launches += 1;
+    if (p.splits > 1) {
+        FS_CUDA(s, fs::launch_attn_combine(p, s->stream));
+        s->launches += 1;
+    }
+    return FS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame, int text_len, int H, int Hkv,
+                     int d, float rope_base) {
+    if (!out) return fail(nullptr, FS_ERR_ARG, "out is NULL");
+    *out = nullptr;
+    if (views < 1 || frames < 1 || tok_per_frame < 1 || text_len < 0)
+        return fail(nullptr, FS_ERR_ARG, "window sizes must be positive (text_len >= 0)");
+    if (H < 1 || Hkv < 1 || H % Hkv) return fail(nullptr, FS_ERR_ARG, "need H, Hkv >= 1 and H %% Hkv == 0");
+    const int G = H / Hkv;
+    if (fs::kTileRows % G) return fail(nullptr, FS_ERR_ARG, "H/Hkv must divide 128 (got %d)", G);
+    if (d != 64 && d != 128) return fail(nullptr, FS_ERR_ARG, "head dim must be 64 or 128 (got %d)", d);
+    if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return fail(nullptr, FS_ERR_ARG, "rope_base must be > 0");
+    const long long ring = (long long)views * frames * tok_per_frame;
+    const long long L = ring + text_len;
+    if (L + fs::kMaxVerify > (long long)fs::kMaxKeyTiles * fs::kTileRows)
+        return fail(nullptr, FS_ERR_ARG, "window too long: L + %d must be <= %d", fs::kMaxVerify,
+                    fs::kMaxKeyTiles * fs::kTileRows);
+
+    fs_stream* s = new (std::nothrow) fs_stream();
+    if (!s) return fail(nullptr, FS_ERR_OOM, "host allocation failed");
+    s->V = views;
+    s->T = frames;
+    s->n = tok_per_frame;
+    s->X = text_len;
+    s->H = H;
+    s->Hkv = Hkv;
+    s->G = G;
+    s->d = d;
+    s->base = rope_base;
+    s->ring_rows = int(ring);
+    s->L = int(L);
+    s->step_tokens = views * tok_per_frame + text_len;
+    s->rows_cap = int(L) + fs::kMaxVerify;
+    s->rope_rows = s->rows_cap;
+    s->slot_frame.assign(frames, -1);
+    if (const char* e = std::getenv("FS_WAIT_LIMIT_NS")) s->wait_limit_ns = std::strtoull(e, nullptr, 10);
+
+    auto bail = [&](int code) {
+        free_all(s);
+        delete s;
+        return code;
+    };
+    cudaError_t e = cudaGetDevice(&s->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&s->num_sms, cudaDevAttrMultiProcessorCount, s->device);
+    if (e != cudaSuccess) return bail(fail(nullptr, FS_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e)));
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, s->device);
+    if (major != 10) return bail(fail(nullptr, FS_ERR_CUDA, "needs an sm_100 GPU (B200); found major %d", major));
+
+    const size_t cache = size_t(Hkv) * s->rows_cap * d * 2;
+    const size_t rope = size_t(s->rope_rows) * (d / 2) * sizeof(float2);
+    s->part_rows_cap = 2 * s->num_sms;
+    const size_t part_o = size_t(s->part_rows_cap) * fs::kTileRows * d * sizeof(float);
+    const size_t part_ml = size_t(s->part_rows_cap) * fs::kTileRows * sizeof(float2);
+    if (cudaMalloc(&s->K_cache, cache) != cudaSuccess || cudaMalloc(&s->V_cache, cache) != cudaSuccess ||
+        cudaMalloc(&s->rope, rope) != cudaSuccess || cudaMalloc(&s->err, sizeof(unsigned)) != cudaSuccess ||
+        cudaMalloc(&s->part_o, part_o) != cudaSuccess || cudaMalloc(&s->part_ml, part_ml) != cudaSuccess) {
+        cudaGetLastError();
+        return bail(fail(nullptr, FS_ERR_OOM, "device allocation of %zu bytes failed", 2 * cache + rope + part_o));
+    }
+    s->cache_bytes = (long long)(2 * cache + rope + part_o + part_ml + sizeof(unsigned));
+    if (cudaMemset(s->K_cache, 0, cache) != cudaSuccess || cudaMemset(s->V_cache, 0, cache) != cudaSuccess ||
+        cudaMemset(s->err, 0, sizeof(unsigned)) != cudaSuccess)
+        return bail(fail(nullptr, FS_ERR_CUDA, "cudaMemset failed"));
+
+    // RoPE table: cos/sin of pos * base^(-2i/d), evaluated in double, stored as float.
+    std::vector<float2> tab(size_t(s->rope_rows) * (d / 2));
+    for (int pos = 0; pos < s->rope_rows; ++pos)
+        for (int i = 0; i < d / 2; ++i) {
+            const double theta = std::pow(double(rope_base), -2.0 * i / d);
+            const double a = double(pos) * theta;
+            tab[size_t(pos) * (d / 2) + i] = make_float2(float(std::cos(a)), float(std::sin(a)));
+        }
+    if (cudaMemcpy(s->rope, tab.data(), rope, cudaMemcpyHostToDevice) != cudaSuccess)
+        return bail(fail(nullptr, FS_ERR_CUDA, "RoPE table upload failed"));
+
+    const uint64_t row_bytes = uint64_t(d) * 2;
+    int rc = make_map(nullptr, &s->tmap_k, s->K_cache, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
+                      fs::kTileRows, 1);
+    if (!rc) rc = make_map(nullptr, &s->tmap_v, s->V_cache, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
+                           fs::kTileRows, 1);
+    if (rc) return bail(rc);
+    *out = s;
+    return FS_OK;
+}
+
+int fs_stream_destroy(fs_stream_t s) {
+    if (!s) return FS_OK;
+    cudaStreamSynchronize(s->stream);
+    free_all(s);
+    delete s;
+    return FS_OK;
+}
+
+int fs_stream_set_stream(fs_stream_t s, void* cuda_stream) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    s->stream = static_cast<cudaStream_t>(cuda_stream);
+    return FS_OK;
+}
+
+int fs_stream_reset(fs_stream_t s) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    s->state = FS_STATE_EXPECT_PREFILL;
+    s->head = 0;
+    s->steps = 0;
+    s->slot_frame.assign(s->T, -1);
+    return FS_OK;
+}
+
+int fs_stream_insert(fs_stream_t s, const void* K_new, const void* V_new) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (!K_new || !V_new) return fail(s, FS_ERR_ARG, "K_new/V_new is NULL");
+    if (!aligned16(K_new) || !aligned16(V_new)) return fail(s, FS_ERR_ARG, "K_new/V_new must be 16-byte aligned");
+    if (s->state == FS_STATE_EXPECT_PREFILL) {
+        s->head = 0;
+        int rc = do_insert(s, K_new, V_new, s->L, 0);
+        if (rc) return rc;
+        for (int f = 0; f < s->T; ++f) s->slot_frame[f] = f;
+        s->state = FS_STATE_PREFILLED;
+        s->last_insert_tokens = s->L;
+        return FS_OK;
+    }
+    int rc = do_insert(s, K_new, V_new, s->step_tokens, 1);
+    if (rc) return rc;
+    s->slot_frame[s->head] = (long long)s->T + s->steps;  // the k-th step inserts frame T-1+k
+    s->head = (s->head + 1) % s->T;
+    s->steps += 1;
+    s->state = FS_STATE_STREAMING;
+    s->last_insert_tokens = s->step_tokens;
+    return FS_OK;
+}
+
+int fs_stream_attend(fs_stream_t s, const void* Q, void* out) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (!Q || !out) return fail(s, FS_ERR_ARG, "Q/out is NULL");
+    if (!aligned16(Q) || !aligned16(out)) return fail(s, FS_ERR_ARG, "Q/out must be 16-byte aligned");
+    if (Q == out) return fail(s, FS_ERR_ARG, "out must not alias Q");
+    if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "attend before the first insert");
+    const bool pre = s->state == FS_STATE_PREFILLED;
+    return do_attend(s, Q, out, pre ? s->L : s->step_tokens, pre ? fs::kQueryPrefill : fs::kQueryStep, s->L);
+}
+
+int fs_stream_attend_ext(fs_stream_t s, const void* Q_x, const void* K_x, const void* V_x, int n_x, void* out) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (!Q_x || !K_x || !V_x || !out) return fail(s, FS_ERR_ARG, "NULL tensor pointer");
+    if (!aligned16(Q_x) || !aligned16(K_x) || !aligned16(V_x) || !aligned16(out))
+        return fail(s, FS_ERR_ARG, "pointers must be 16-byte aligned");
+    if (n_x < 1 || n_x > FS_MAX_VERIFY_TOKENS) return fail(s, FS_ERR_ARG, "n_x must be in [1, %d]", FS_MAX_VERIFY_TOKENS);
+    if (Q_x == out) return fail(s, FS_ERR_ARG, "out must not alias Q_x");
+    if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "verify before the first insert");
+    int rc = do_insert(s, K_x, V_x, n_x, 2);
+    if (rc) return rc;
+    return do_attend(s, Q_x, out, n_x, fs::kQueryVerify, s->L + n_x);
+}
+
+int fs_stream_step_host(fs_stream_t s, const void* K_new_h, const void* V_new_h, const void* Q_h, void* out_h) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (!K_new_h || !V_new_h || !Q_h || !out_h) return fail(s, FS_ERR_ARG, "NULL host pointer");
+    const int nt = s->state == FS_STATE_EXPECT_PREFILL ? s->L : s->step_tokens;
+    const size_t kv = size_t(nt) * s->Hkv * s->d * 2;
+    const size_t qb = size_t(nt) * s->H * s->d * 2;  // Q, bf16
+    const size_t ob = 2 * qb;                           // out, fp32
+    const size_t need = 2 * kv + qb + ob + 4 * 256;
+    if (need > s->stage_bytes) {
+        // Grown on first use (sized for the largest call so far), outside any capture.
+        FS_CUDA(s, cudaStreamSynchronize(s->stream));
+        cudaFree(s->stage);
+        s->stage = nullptr;
+        s->stage_bytes = 0;
+        if (cudaMalloc(&s->stage, need) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(s, FS_ERR_OOM, "staging allocation of %zu bytes failed", need);
+        }
+        s->stage_bytes = need;
+    }
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    char* base = static_cast<char*>(s->stage);
+    void* dK = base;
+    void* dV = base + up(kv);
+    void* dQ = base + 2 * up(kv);
+    void* dO = base + 2 * up(kv) + up(qb);
+    FS_CUDA(s, cudaMemcpyAsync(dK, K_new_h, kv, cudaMemcpyHostToDevice, s->stream));
+    FS_CUDA(s, cudaMemcpyAsync(dV, V_new_h, kv, cudaMemcpyHostToDevice, s->stream));
+    FS_CUDA(s, cudaMemcpyAsync(dQ, Q_h, qb, cudaMemcpyHostToDevice, s->stream));
+    int rc = fs_stream_insert(s, dK, dV);
+    if (rc) return rc;
+    rc = fs_stream_attend(s, dQ, dO);
+    if (rc) return rc;
+    FS_CUDA(s, cudaMemcpyAsync(out_h, dO, ob, cudaMemcpyDeviceToHost, s->stream));
+    return FS_OK;
+}
+
+int fs_stream_sync(fs_stream_t s) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    FS_CUDA(s, cudaStreamSynchronize(s->stream));
+    return check_err_word(s);
+}
+
+int fs_stream_info(fs_stream_t s, fs_stream_info_t* info) {
+    if (!s || !info) return fail(s, FS_ERR_ARG, "NULL argument");
+    info->views = s->V;
+    info->frames = s->T;
+    info->tok_per_frame = s->n;
+    info->text_len = s->X;
+    info->H = s->H;
+    info->Hkv = s->Hkv;
+    info->d = s->d;
+    info->window_len = s->L;
+    info->step_tokens = s->step_tokens;
+    info->state = s->state;
+    info->insert_tokens = s->state == FS_STATE_EXPECT_PREFILL ? s->L : s->step_tokens;
+    info->query_tokens = s->state == FS_STATE_EXPECT_PREFILL ? 0 : (s->state == FS_STATE_PREFILLED ? s->L : s->step_tokens);
+    info->head = s->head;
+    info->steps = s->steps;
+    info->cache_bytes = s->cache_bytes;
+    info->launches = s->launches;
+    return FS_OK;
+}
+
+int fs_stream_debug_export(fs_stream_t s, void* K_phys, void* V_phys, int32_t* pos_phys, int32_t* frame_id_phys) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "nothing inserted yet");
+    FS_CUDA(s, cudaStreamSynchronize(s->stream));
+    const int rows = s->L;
+    const size_t row_bytes = size_t(s->d) * 2;
+    for (int h = 0; h < s->Hkv; ++h) {
+        const size_t src = size_t(h) * s->rows_cap * row_bytes;
+        const size_t dst = size_t(h) * rows * row_bytes;
+        if (K_phys)
+            FS_CUDA(s, cudaMemcpy(static_cast<char*>(K_phys) + dst, reinterpret_cast<char*>(s->K_cache) + src,
+                                  rows * row_bytes, cudaMemcpyDeviceToHost));
+        if (V_phys)
+            FS_CUDA(s, cudaMemcpy(static_cast<char*>(V_phys) + dst, reinterpret_cast<char*>(s->V_cache) + src,
+                                  rows * row_bytes, cudaMemcpyDeviceToHost));
+    }
+    if (pos_phys) {
+        // Positions as the attention kernel derives them (same device function).
+        int* dpos = nullptr;
+        FS_CUDA(s, cudaMalloc(&dpos, size_t(rows) * sizeof(int)));
+        cudaError_t e = fs::launch_positions(shape_of(s), rows, dpos, s->stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s->stream);
+        if (e == cudaSuccess) e = cudaMemcpy(pos_phys, dpos, size_t(rows) * sizeof(int), cudaMemcpyDeviceToHost);
+        cudaFree(dpos);
+        if (e != cudaSuccess) return fail(s, FS_ERR_CUDA, "position export failed: %s", cudaGetErrorString(e));
+    }
+    if (frame_id_phys) {
+        for (int r = 0; r < rows; ++r) {
+            if (r >= s->ring_rows) {
+                frame_id_phys[r] = -1;
+            } else {
+                const int slot = (r % (s->T * s->n)) / s->n;
+                frame_id_phys[r] = int32_t(s->slot_frame[slot]);
+            }
+        }
+    }
+    return check_err_word(s);
+}
+
+int fs_stream_debug_wait_probe(fs_stream_t s, int limit_us) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (limit_us < 1 || limit_us > 1000000) return fail(s, FS_ERR_ARG, "limit_us must be in [1, 1e6]");
+    FS_CUDA(s, fs::launch_wait_probe(s->err, (unsigned long long)limit_us * 1000ull, s->stream));
+    return fs_stream_sync(s);
+}
+
+const char* fs_stream_last_error(fs_stream_t s) { return s ? s->last_error.c_str() : g_last_error.c_str(); }
+
+const char* fs_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"
