@@ -89,28 +89,37 @@ def recorded_traffic(workload_id):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling while the timed region runs."""
+    """nvidia-smi clock/throttle sampling; only samples taken inside the timed
+    window (host wall-clock marks) are summarised."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index):
-        self.idx = device_index
+    def __init__(self, gpu):
+        self.gpu = gpu
         self.proc = None
+        self.t0 = self.t1 = None
+        self.lines = []
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(1.0)  # let nvidia-smi start sampling before the timed region
         except Exception:
             self.proc = None
-        return self
 
-    def __exit__(self, *a):
-        self.lines = []
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
         if self.proc is not None:
+            time.sleep(0.05)
             self.proc.terminate()
             try:
                 out, _ = self.proc.communicate(timeout=5)
@@ -120,25 +129,33 @@ class ClockSampler:
             self.lines = [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        import datetime
+
+        sm, mx, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        for l in self.lines:
             f = [x.strip() for x in l.split(",")]
             if len(f) < 9:
                 continue
             try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            if self.t0 is None or not (self.t0 - 0.02 <= ts <= self.t1 + 0.02):
+                continue
+            try:
                 sm.append(float(f[1]))
                 mx = float(f[2])
+                power.append(float(f[3]))
             except ValueError:
                 continue
             for name, val in zip(names, f[5:9]):
                 if val.lower() == "active":
                     reasons.add(name)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["no samples"]}
-        load = sorted(sm)[len(sm) // 4:] or sm  # drop the idle lead-in samples
-        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["no samples inside the timed region"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
 
 
 def gpu_id(dev):
@@ -276,6 +293,8 @@ def run_ours(args):
             if ev is not None:
                 ev[l][2].record(stream)
 
+    clk = ClockSampler(gpu_id(dev))
+    clk.start()
     for k in range(args.warmup):
         step(k)
     torch.cuda.synchronize()
@@ -283,12 +302,14 @@ def run_ours(args):
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(layers)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
-    with ClockSampler(gpu_id(dev)) as clk:
-        start.record(stream)
-        for k in range(args.steps):
-            step(args.warmup + k, evs[k])
-        end.record(stream)
-        torch.cuda.synchronize()
+    clk.mark_start()
+    start.record(stream)
+    for k in range(args.steps):
+        step(args.warmup + k, evs[k])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk.mark_end()
+    clk.stop()
     barrier(world)
     launches = sum(s.info().launches for s in streams) - launches0
     elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
@@ -450,7 +471,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=3)

@@ -90,11 +90,25 @@ struct InsertParams {
     int V, T, n, X, ring_rows, head;
 };
 
+struct RopeParams {
+    WindowShape w;
+    int key_rows;         // rows per kv head to rotate
+    int Hkv, d;
+    const float2* rope;   // [rope_rows][d/2] (cos, sin)
+    unsigned* err;
+    unsigned long long wait_limit_ns;
+};
+
 // Launchers (defined in the .cu files); all enqueue on `stream` and return the
 // launch's cudaError_t.
 cudaError_t launch_kv_stream_insert(const InsertParams& p, int num_sms, cudaStream_t stream);
-cudaError_t launch_stream_attn(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tk,
-                               const CUtensorMap& tv, cudaStream_t stream);
+// kv_stream_rope: bf16 cache (tk, tv) -> fp16 rotated K hi (tkh), lo (tkl) and V (tv16).
+cudaError_t launch_kv_stream_rope(const RopeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                                  const CUtensorMap& tkh, const CUtensorMap& tkl, const CUtensorMap& tv16,
+                                  cudaStream_t stream);
+// stream_attn over the rotated operand cache (tkh, tkl, tv16).
+cudaError_t launch_stream_attn(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tkh,
+                               const CUtensorMap& tkl, const CUtensorMap& tv16, cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_positions(const WindowShape& w, int rows, int* pos_out, cudaStream_t stream);
 cudaError_t launch_wait_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);

@@ -34,8 +34,11 @@ struct fs_stream {
     std::vector<long long> slot_frame;  // frame id held by each ring slot (same for all views)
     cudaStream_t stream = nullptr;
     int device = 0, num_sms = 148;
-    uint16_t* K_cache = nullptr;
+    uint16_t* K_cache = nullptr;  // pre-RoPE bf16 ring + text + drafted-block rows
     uint16_t* V_cache = nullptr;
+    uint16_t* Kh = nullptr;       // per-step operands: rotated K fp16 hi / lo, V fp16
+    uint16_t* Kl = nullptr;
+    uint16_t* V16 = nullptr;
     float2* rope = nullptr;
     unsigned* err = nullptr;
     float* part_o = nullptr;
@@ -43,7 +46,7 @@ struct fs_stream {
     int part_rows_cap = 0;  // rows of 128 query rows x d fp32 the split scratch holds
     void* stage = nullptr;  // host-path staging: K, V, Q, out
     size_t stage_bytes = 0;
-    CUtensorMap tmap_k, tmap_v;
+    CUtensorMap tmap_k, tmap_v, tmap_kh, tmap_kl, tmap_v16;
     unsigned long long wait_limit_ns = 2000000000ull;
     long long cache_bytes = 0;
     long long launches = 0;
@@ -84,16 +87,17 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// 3-D bf16 tensor map, 128-byte swizzle, box {64, b1, b2}, out-of-range reads as zero.
+// 3-D 16-bit tensor map, 128-byte swizzle, box {64, b1, b2}, out-of-range reads as zero.
 int make_map(fs_stream_t s, CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-             uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b1, uint32_t b2) {
+             uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b1, uint32_t b2,
+             CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     auto enc = get_encode();
     if (!enc) return fail(s, FS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
     cuuint64_t dims[3] = {d0, d1, d2};
     cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
     cuuint32_t box[3] = {64, b1, b2};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = enc(m, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(s, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
@@ -116,6 +120,9 @@ WindowShape shape_of(const fs_stream* s) {
 void free_all(fs_stream* s) {
     cudaFree(s->K_cache);
     cudaFree(s->V_cache);
+    cudaFree(s->Kh);
+    cudaFree(s->Kl);
+    cudaFree(s->V16);
     cudaFree(s->rope);
     cudaFree(s->err);
     cudaFree(s->part_o);
@@ -188,7 +195,18 @@ int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key
     p.part_ml = s->part_ml;
     p.err = s->err;
     p.wait_limit_ns = s->wait_limit_ns;
-    FS_CUDA(s, fs::launch_stream_attn(p, static_cast<const uint16_t*>(Q), s->tmap_k, s->tmap_v, s->stream));
+    fs::RopeParams rp;
+    rp.w = p.w;
+    rp.key_rows = key_rows;
+    rp.Hkv = s->Hkv;
+    rp.d = s->d;
+    rp.rope = s->rope;
+    rp.err = s->err;
+    rp.wait_limit_ns = s->wait_limit_ns;
+    FS_CUDA(s, fs::launch_kv_stream_rope(rp, s->tmap_k, s->tmap_v, s->tmap_kh, s->tmap_kl, s->tmap_v16, s->stream));
+    s->launches += 1;
+    FS_CUDA(s, fs::launch_stream_attn(p, static_cast<const uint16_t*>(Q), s->tmap_kh, s->tmap_kl, s->tmap_v16,
+                                      s->stream));
     s->launches += 1;
     if (p.splits > 1) {
         FS_CUDA(s, fs::launch_attn_combine(p, s->stream));
@@ -255,12 +273,14 @@ int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame,
     const size_t part_o = size_t(s->part_rows_cap) * fs::kTileRows * d * sizeof(float);
     const size_t part_ml = size_t(s->part_rows_cap) * fs::kTileRows * sizeof(float2);
     if (cudaMalloc(&s->K_cache, cache) != cudaSuccess || cudaMalloc(&s->V_cache, cache) != cudaSuccess ||
+        cudaMalloc(&s->Kh, cache) != cudaSuccess || cudaMalloc(&s->Kl, cache) != cudaSuccess ||
+        cudaMalloc(&s->V16, cache) != cudaSuccess ||
         cudaMalloc(&s->rope, rope) != cudaSuccess || cudaMalloc(&s->err, sizeof(unsigned)) != cudaSuccess ||
         cudaMalloc(&s->part_o, part_o) != cudaSuccess || cudaMalloc(&s->part_ml, part_ml) != cudaSuccess) {
         cudaGetLastError();
-        return bail(fail(nullptr, FS_ERR_OOM, "device allocation of %zu bytes failed", 2 * cache + rope + part_o));
+        return bail(fail(nullptr, FS_ERR_OOM, "device allocation of %zu bytes failed", 5 * cache + rope + part_o));
     }
-    s->cache_bytes = (long long)(2 * cache + rope + part_o + part_ml + sizeof(unsigned));
+    s->cache_bytes = (long long)(5 * cache + rope + part_o + part_ml + sizeof(unsigned));
     if (cudaMemset(s->K_cache, 0, cache) != cudaSuccess || cudaMemset(s->V_cache, 0, cache) != cudaSuccess ||
         cudaMemset(s->err, 0, sizeof(unsigned)) != cudaSuccess)
         return bail(fail(nullptr, FS_ERR_CUDA, "cudaMemset failed"));
@@ -281,6 +301,13 @@ int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame,
                       fs::kTileRows, 1);
     if (!rc) rc = make_map(nullptr, &s->tmap_v, s->V_cache, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
                            fs::kTileRows, 1);
+    const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!rc) rc = make_map(nullptr, &s->tmap_kh, s->Kh, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
+                           fs::kTileRows, 1, f16);
+    if (!rc) rc = make_map(nullptr, &s->tmap_kl, s->Kl, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
+                           fs::kTileRows, 1, f16);
+    if (!rc) rc = make_map(nullptr, &s->tmap_v16, s->V16, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
+                           fs::kTileRows, 1, f16);
     if (rc) return bail(rc);
     *out = s;
     return FS_OK;

@@ -11,6 +11,7 @@
 // Work: a pure copy, bound by HBM bandwidth. Each thread moves 16-byte chunks;
 // consecutive threads take consecutive chunks of the token-major source, so
 // loads are fully coalesced and stores form 256-byte runs (one d=128 vector).
+// All index arithmetic is 32-bit (a step moves < 2^31 chunks).
 #include "fs_internal.cuh"
 
 namespace fs {
@@ -18,7 +19,7 @@ namespace fs {
 namespace {
 
 constexpr int kInsertThreads = 256;
-constexpr int kInsertUnroll = 4;
+constexpr int kTokensPerBlock = 4;
 
 __device__ __forceinline__ int dest_row(const InsertParams& p, int t) {
     if (p.mode == 0) return t;                                   // prefill: window order, head = slot 0
@@ -32,45 +33,35 @@ __device__ __forceinline__ int dest_row(const InsertParams& p, int t) {
     return p.ring_rows + (t - vn);                               // fresh text
 }
 
+// One block moves kTokensPerBlock tokens: their Hkv x chunks 16-byte chunks of
+// K and of V. Source reads are contiguous; each (token, kv head) vector lands
+// as one contiguous run of d*2 bytes in its kv head's ring.
 __global__ void __launch_bounds__(kInsertThreads) kv_stream_insert_kernel(const InsertParams p) {
-    const long long total = (long long)p.N * p.Hkv * p.chunks;
-    const long long stride = (long long)gridDim.x * kInsertThreads * kInsertUnroll;
-    for (long long base = (long long)blockIdx.x * kInsertThreads * kInsertUnroll + threadIdx.x; base < total;
-         base += stride) {
-        uint4 k[kInsertUnroll], v[kInsertUnroll];
-#pragma unroll
-        for (int u = 0; u < kInsertUnroll; ++u) {
-            const long long idx = base + (long long)u * kInsertThreads;
-            if (idx < total) {
-                k[u] = __ldcs(p.K_src + idx);   // streamed once: do not keep in L1/L2
-                v[u] = __ldcs(p.V_src + idx);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kInsertUnroll; ++u) {
-            const long long idx = base + (long long)u * kInsertThreads;
-            if (idx < total) {
-                const int c = int(idx % p.chunks);
-                const long long th = idx / p.chunks;
-                const int h = int(th % p.Hkv);
-                const int t = int(th / p.Hkv);
-                const long long dst = ((long long)h * p.rows_cap + dest_row(p, t)) * p.chunks + c;
-                p.K_cache[dst] = k[u];
-                p.V_cache[dst] = v[u];
-            }
-        }
+    const int per_tok = p.Hkv * p.chunks;
+    const int t0 = blockIdx.x * kTokensPerBlock;
+    const int nt = min(kTokensPerBlock, p.N - t0);
+    const int total = nt * per_tok;
+    const size_t src0 = (size_t)t0 * per_tok;
+    for (int i = threadIdx.x; i < total; i += kInsertThreads) {
+        const int tl = i / per_tok;
+        const int hc = i - tl * per_tok;
+        const int h = hc / p.chunks;
+        const int c = hc - h * p.chunks;
+        const uint4 k = __ldcs(p.K_src + src0 + i);  // streamed once: do not keep in L1
+        const uint4 v = __ldcs(p.V_src + src0 + i);
+        const size_t dst = ((size_t)h * p.rows_cap + dest_row(p, t0 + tl)) * p.chunks + c;
+        p.K_cache[dst] = k;
+        p.V_cache[dst] = v;
     }
 }
 
 }  // namespace
 
 cudaError_t launch_kv_stream_insert(const InsertParams& p, int num_sms, cudaStream_t stream) {
-    const long long total = (long long)p.N * p.Hkv * p.chunks;
-    if (total <= 0) return cudaSuccess;
-    long long blocks = (total + kInsertThreads * kInsertUnroll - 1) / (kInsertThreads * kInsertUnroll);
-    const long long cap = (long long)num_sms * 8;  // 8 resident 256-thread blocks per SM
-    if (blocks > cap) blocks = cap;
-    kv_stream_insert_kernel<<<(unsigned)blocks, kInsertThreads, 0, stream>>>(p);
+    (void)num_sms;
+    if (p.N <= 0) return cudaSuccess;
+    const unsigned blocks = unsigned((p.N + kTokensPerBlock - 1) / kTokensPerBlock);
+    kv_stream_insert_kernel<<<blocks, kInsertThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

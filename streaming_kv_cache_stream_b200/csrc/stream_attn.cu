@@ -9,18 +9,21 @@
 //
 // One CTA = one (kv head, 128-row query tile[, key split]). A query tile packs
 // 128/G tokens x the G query heads that share the kv head, so every key tile
-// is loaded and rotated once for all G heads (GQA). Warp roles, 12 warps:
-//   warp 0      TMA producer: K and V tiles, two stages each;
+// is loaded once for all G heads (GQA). The keys were rotated once for this
+// step by kv_stream_rope (RoPE in shared memory at their shifted positions,
+// written as fp16 hi + lo, V as fp16); this kernel rotates its query rows.
+// Warp roles, 12 warps:
+//   warp 0      TMA producer: K hi + K lo tile and V tile, two stages each;
 //   warp 1      TMEM allocator and tcgen05.mma issuer (one thread);
 //   warps 4-7   softmax: one query row per thread; S read from TMEM, streaming
 //               mask, online softmax in fp32 with exp2, P written back into
 //               TMEM over S, lazy rescale of O in TMEM, epilogue;
-//   warps 8-11  RoPE: rotate-half rotation of the query rows (into TMEM) and of
-//               each K tile in place in shared memory; V tiles to fp16.
+//   warps 8-11  RoPE of the query rows at their window positions, written into
+//               TMEM as the A operand (fp16 hi + lo), once per CTA.
 // Pipeline per key tile j (S double-buffered in TMEM):
-//   TMA K_j,V_j -> RoPE(K_j), V_j->fp16 -> MMA S_j = Q K_j^T -> softmax(S_j)
-//   -> P_j -> MMA O += P_j V_j; QK_{j+1} is issued before PV_j, so the tensor
-//   core works on the next tile while the softmax warps run.
+//   TMA K_j, V_j -> MMA S_j = Q K_j^T -> softmax(S_j) -> P_j -> MMA O += P_j V_j;
+//   QK_{j+1} is issued before PV_j, so the tensor core works on the next tile
+//   while the softmax warps run.
 // Key tiles are walked in physical ring order; positions come from key_pos(),
 // so the ring never moves. Tiles whose every key is after the tile's last
 // query are skipped; tiles that are entirely visible skip the elementwise mask.
@@ -31,8 +34,8 @@
 // in fp32 as Q_hi K_hi + Q_hi K_lo + Q_lo K_hi: a single fp16 rounding of the
 // rotated operands (2^-12 relative) moves the softmax weights of competing
 // large-norm keys by ~1e-2 at the 1%-outlier-key workload, the split brings
-// the scores to ~2^-22 relative. P is fp16 (V is converted to fp16 in shared
-// memory to match), O accumulates in fp32, and the output is stored in fp32.
+// the scores to ~2^-22 relative. P is fp16 (V is fp16 to match), O
+// accumulates in fp32, and the output is stored in fp32.
 //
 // Shared-memory tiles use the 128-byte swizzle that TMA writes and tcgen05
 // reads: rows of 128 bytes, 16-byte chunk c of row r at chunk position
@@ -56,9 +59,9 @@ constexpr float kRescaleLog2 = 8.0f;     // rescale O only when the max grows by
 __device__ __forceinline__ constexpr uint32_t col_s(int s) { return s ? 128u : 0u; }
 
 enum : int {
-    kBarQReady = 0, kBarKFull0, kBarKFull1, kBarKRot0, kBarKRot1, kBarKEmpty0, kBarKEmpty1,
-    kBarVFull0, kBarVFull1, kBarVConv0, kBarVConv1, kBarVEmpty0, kBarVEmpty1, kBarSFull0, kBarSFull1,
-    kBarPFull0, kBarPFull1, kBarSFree0, kBarSFree1, kBarOFull, kBarMmaDone, kNumBars
+    kBarQReady = 0, kBarKFull0, kBarKFull1, kBarKEmpty0, kBarKEmpty1, kBarVFull0, kBarVFull1,
+    kBarVEmpty0, kBarVEmpty1, kBarSFull0, kBarSFull1, kBarPFull0, kBarPFull1, kBarSFree0, kBarSFree1,
+    kBarOFull, kBarMmaDone, kNumBars
 };
 
 constexpr uint8_t kSkip = 0, kFull = 1, kPartial = 2;
@@ -111,68 +114,6 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
     lo = pack_f16x2(a - hf.x, b - hf.y);
 }
 
-// Rotate one 128-byte-swizzled key row of a [128 x D] bf16 tile: rotate-half
-// RoPE with (cos, sin) of pos * theta_i in `cs` (i < D/2). The fp16 hi part
-// overwrites the row in place; the lo part goes to the same offsets of the
-// tile at `lo_tile`. Pair (i, i + D/2): for D = 128 the halves are the two
-// 16 KB regions at the same offset; for D = 64 chunks c and c + 4 of the row.
-template <int D>
-__device__ __forceinline__ void rope_key_row(uint8_t* tile, uint8_t* lo_tile, int row,
-                                             const float2* __restrict__ cs) {
-    constexpr int kPairs = D / 16;
-    const int sw = row & 7;
-#pragma unroll
-    for (int c = 0; c < kPairs; ++c) {
-        const int off_a = row * 128 + ((c ^ sw) << 4);
-        const int off_b = D == 128 ? off_a + kRegion : row * 128 + (((c + 4) ^ sw) << 4);
-        const uint4 a = *reinterpret_cast<const uint4*>(tile + off_a);
-        const uint4 b = *reinterpret_cast<const uint4*>(tile + off_b);
-        const float4* t4 = reinterpret_cast<const float4*>(cs + 8 * c);
-        const float4 t0 = __ldg(t4 + 0), t1 = __ldg(t4 + 1), t2 = __ldg(t4 + 2), t3 = __ldg(t4 + 3);
-        const float co[8] = {t0.x, t0.z, t1.x, t1.z, t2.x, t2.z, t3.x, t3.z};
-        const float si[8] = {t0.y, t0.w, t1.y, t1.w, t2.y, t2.w, t3.y, t3.w};
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-        uint32_t ah[4], al[4], bh[4], bl[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float x0 = bf16lo(aw[q]), x1 = bf16hi(aw[q]);
-            const float y0 = bf16lo(bw[q]), y1 = bf16hi(bw[q]);
-            const float c0 = co[2 * q], s0 = si[2 * q], c1 = co[2 * q + 1], s1 = si[2 * q + 1];
-            split2(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1, ah[q], al[q]);
-            split2(y0 * c0 + x0 * s0, y1 * c1 + x1 * s1, bh[q], bl[q]);
-        }
-        *reinterpret_cast<uint4*>(tile + off_a) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
-        *reinterpret_cast<uint4*>(tile + off_b) = make_uint4(bh[0], bh[1], bh[2], bh[3]);
-        *reinterpret_cast<uint4*>(lo_tile + off_a) = make_uint4(al[0], al[1], al[2], al[3]);
-        *reinterpret_cast<uint4*>(lo_tile + off_b) = make_uint4(bl[0], bl[1], bl[2], bl[3]);
-    }
-}
-
-template <int D>
-__device__ __forceinline__ void zero_key_row(uint8_t* tile, uint8_t* lo_tile, int row) {
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        const int off = (c >> 3) * kRegion + row * 128 + ((c & 7) << 4);
-        *reinterpret_cast<uint4*>(tile + off) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(lo_tile + off) = make_uint4(0, 0, 0, 0);
-    }
-}
-
-// bf16 -> fp16 in place for one row of a [128 x D] tile (elementwise, so the
-// swizzle only spreads the row's chunks over the banks).
-template <int D>
-__device__ __forceinline__ void v_row_to_f16(uint8_t* tile, int row) {
-    const int sw = row & 7;
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        uint4* q = reinterpret_cast<uint4*>(tile + (c >> 3) * kRegion + row * 128 + (((c & 7) ^ sw) << 4));
-        const uint4 v = *q;
-        *q = make_uint4(pack_f16x2(bf16lo(v.x), bf16hi(v.x)), pack_f16x2(bf16lo(v.y), bf16hi(v.y)),
-                        pack_f16x2(bf16lo(v.z), bf16hi(v.z)), pack_f16x2(bf16lo(v.w), bf16hi(v.w)));
-    }
-}
-
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
                  "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
@@ -186,28 +127,49 @@ template <int D>
 __device__ __forceinline__ void rope_query_row(const uint16_t* __restrict__ qrow, const float2* __restrict__ cs,
                                                float scale, uint32_t t_hi, uint32_t t_lo) {
     constexpr int kHalf = D / 2;
+    constexpr int kM = kHalf / 16;  // 16-element blocks per half
 #pragma unroll
-    for (int m = 0; m < kHalf / 16; ++m) {
-        // elements [16m, 16m+16) and their partners [kHalf + 16m, ...)
-        const uint4* pa = reinterpret_cast<const uint4*>(qrow + 16 * m);
-        const uint4* pb = reinterpret_cast<const uint4*>(qrow + kHalf + 16 * m);
-        const uint4 a0 = __ldg(pa), a1 = __ldg(pa + 1), b0 = __ldg(pb), b1 = __ldg(pb + 1);
-        const uint32_t aw[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        const float4* t4 = reinterpret_cast<const float4*>(cs + 16 * m);
-        uint32_t ah[8], al[8], bh[8], bl[8];
+    for (int m0 = 0; m0 < kM; m0 += 2) {
+        // Issue every load of two blocks before any arithmetic: one round trip per pair.
+        uint4 qa[2][2], qb[2][2];
+        float4 tt[2][8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float4 t = __ldg(t4 + q);  // (cos, sin) of elements 16m + 2q, 16m + 2q + 1
-            const float x0 = bf16lo(aw[q]), x1 = bf16hi(aw[q]);
-            const float y0 = bf16lo(bw[q]), y1 = bf16hi(bw[q]);
-            split2((x0 * t.x - y0 * t.y) * scale, (x1 * t.z - y1 * t.w) * scale, ah[q], al[q]);
-            split2((y0 * t.x + x0 * t.y) * scale, (y1 * t.z + x1 * t.w) * scale, bh[q], bl[q]);
+        for (int u = 0; u < 2; ++u) {
+            const int m = m0 + u;
+            if (m < kM) {
+                const uint4* pa = reinterpret_cast<const uint4*>(qrow + 16 * m);
+                const uint4* pb = reinterpret_cast<const uint4*>(qrow + kHalf + 16 * m);
+                qa[u][0] = __ldg(pa);
+                qa[u][1] = __ldg(pa + 1);
+                qb[u][0] = __ldg(pb);
+                qb[u][1] = __ldg(pb + 1);
+                const float4* t4 = reinterpret_cast<const float4*>(cs + 16 * m);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) tt[u][q] = __ldg(t4 + q);
+            }
         }
-        tmem_st8(t_hi + 8 * m, ah);
-        tmem_st8(t_hi + kHalf / 2 + 8 * m, bh);
-        tmem_st8(t_lo + 8 * m, al);
-        tmem_st8(t_lo + kHalf / 2 + 8 * m, bl);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int m = m0 + u;
+            if (m >= kM) break;
+            const uint32_t aw[8] = {qa[u][0].x, qa[u][0].y, qa[u][0].z, qa[u][0].w,
+                                    qa[u][1].x, qa[u][1].y, qa[u][1].z, qa[u][1].w};
+            const uint32_t bw[8] = {qb[u][0].x, qb[u][0].y, qb[u][0].z, qb[u][0].w,
+                                    qb[u][1].x, qb[u][1].y, qb[u][1].z, qb[u][1].w};
+            uint32_t ah[8], al[8], bh[8], bl[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 t = tt[u][q];  // (cos, sin) of elements 16m + 2q, 16m + 2q + 1
+                const float x0 = bf16lo(aw[q]), x1 = bf16hi(aw[q]);
+                const float y0 = bf16lo(bw[q]), y1 = bf16hi(bw[q]);
+                split2((x0 * t.x - y0 * t.y) * scale, (x1 * t.z - y1 * t.w) * scale, ah[q], al[q]);
+                split2((y0 * t.x + x0 * t.y) * scale, (y1 * t.z + x1 * t.w) * scale, bh[q], bl[q]);
+            }
+            tmem_st8(t_hi + 8 * m, ah);
+            tmem_st8(t_hi + kHalf / 2 + 8 * m, bh);
+            tmem_st8(t_lo + 8 * m, al);
+            tmem_st8(t_lo + kHalf / 2 + 8 * m, bl);
+        }
     }
 }
 
@@ -228,7 +190,8 @@ __device__ __forceinline__ bool vote_all_ok_wg(bool ok) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     stream_attn_kernel(const __grid_constant__ AttnParams p, const uint16_t* __restrict__ Q,
-                       const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+                       const __grid_constant__ CUtensorMap tkh, const __grid_constant__ CUtensorMap tkl,
+                       const __grid_constant__ CUtensorMap tv16) {
     using L = Layout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -256,10 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar(kBarQReady), 128);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(kBarKFull0 + s), 1);
-            mbar_init(bar(kBarKRot0 + s), 128);
             mbar_init(bar(kBarKEmpty0 + s), 1);
             mbar_init(bar(kBarVFull0 + s), 1);
-            mbar_init(bar(kBarVConv0 + s), 128);
             mbar_init(bar(kBarVEmpty0 + s), 1);
             mbar_init(bar(kBarSFull0 + s), 1);
             mbar_init(bar(kBarPFull0 + s), 128);
@@ -313,30 +274,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Register split, one setmaxnreg per warpgroup at the head of its region: the
     // softmax warpgroup holds a 128-column S row per thread.
-    // 128 x 232 + 256 x 128 = 62464 <= 384 x 168 registers allocated at launch.
+    // 128 x (80 + 232 + 192) <= 384 x 168, the registers allocated at launch.
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 128;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
         if (warp == 0) {
             // ============================================= TMA producer
             if (lane == 0 && nt > 0) {
-                tma_prefetch_desc(&tk);
-                tma_prefetch_desc(&tv);
+                tma_prefetch_desc(&tkh);
+                tma_prefetch_desc(&tkl);
+                tma_prefetch_desc(&tv16);
                 for (int k = 0; k < nt; ++k) {
                     const int s = k & 1;
                     const uint32_t par = ((k >> 1) & 1) ^ 1;
                     const int j = ctrl.list[kbeg + k] & 0x1FFF;
                     if (!wait(bar(kBarKEmpty0 + s), par)) break;
-                    mbar_arrive_expect_tx(bar(kBarKFull0 + s), L::kTileBytes);
+                    mbar_arrive_expect_tx(bar(kBarKFull0 + s), 2 * L::kTileBytes);
                     const uint32_t kd = smem_u32(smem + L::kK0 + s * L::kKStage);
 #pragma unroll
-                    for (int r = 0; r < D / 64; ++r)
-                        tma_load_3d(kd + r * kRegion, &tk, r * 64, j * kTileRows, kvh, bar(kBarKFull0 + s));
+                    for (int r = 0; r < D / 64; ++r) {
+                        tma_load_3d(kd + r * kRegion, &tkh, r * 64, j * kTileRows, kvh, bar(kBarKFull0 + s));
+                        tma_load_3d(kd + L::kTileBytes + r * kRegion, &tkl, r * 64, j * kTileRows, kvh,
+                                    bar(kBarKFull0 + s));
+                    }
                     if (!wait(bar(kBarVEmpty0 + s), par)) break;
                     mbar_arrive_expect_tx(bar(kBarVFull0 + s), L::kTileBytes);
                     const uint32_t vd = smem_u32(smem + L::kV0 + s * L::kTileBytes);
 #pragma unroll
                     for (int r = 0; r < D / 64; ++r)
-                        tma_load_3d(vd + r * kRegion, &tv, r * 64, j * kTileRows, kvh, bar(kBarVFull0 + s));
+                        tma_load_3d(vd + r * kRegion, &tv16, r * 64, j * kTileRows, kvh, bar(kBarVFull0 + s));
                 }
             }
         } else if (warp == 1) {
@@ -349,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int k = 0; ok && k <= nt; ++k) {
                     if (k < nt) {
                         const int s = k & 1;
-                        if (!(ok = wait(bar(kBarKRot0 + s), (k >> 1) & 1))) break;
+                        if (!(ok = wait(bar(kBarKFull0 + s), (k >> 1) & 1))) break;
                         if (k >= 2 && !(ok = wait(bar(kBarSFree0 + s), ((k - 2) >> 1) & 1))) break;
                         tc_fence_after();
                         const uint32_t kh = smem_u32(smem + L::kK0 + s * L::kKStage);
@@ -372,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int s = kp & 1;
                         const uint32_t par = (kp >> 1) & 1;
                         if (!(ok = wait(bar(kBarPFull0 + s), par))) break;
-                        if (!(ok = wait(bar(kBarVConv0 + s), par))) break;
+                        if (!(ok = wait(bar(kBarVFull0 + s), par))) break;
                         tc_fence_after();
                         const uint32_t vs = smem_u32(smem + L::kV0 + s * L::kTileBytes);
 #pragma unroll
@@ -518,41 +483,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.part_ml[part_row] = make_float2(-INFINITY, 0.f);
         }
     } else {
-        // ================================================= RoPE on Q and K, V to fp16
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 128;");
+        // ================================================= RoPE on Q (rows into TMEM)
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 192;");
         const int r = tid - 256;
         if (nt > 0) {
-            {
-                const int t = t0 + r / p.G;
-                const int h = kvh * p.G + r % p.G;
-                // Rows past the last token rotate a valid row (token t0) and are never stored.
-                const int tt = t < t_end ? t : t0;
-                const int qp = query_pos(p.w, p.q_mode, tt);
-                rope_query_row<D>(Q + ((size_t)tt * p.H + h) * D, p.rope + (size_t)qp * (D / 2), p.q_scale,
-                                  tmem + kColQ + lane_off, tmem + kColQ + D / 2 + lane_off);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(kBarQReady));
-            }
-            bool ok = true;
-            for (int k = 0; ok && k < nt; ++k) {
-                const int s = k & 1;
-                const uint32_t par = (k >> 1) & 1;
-                if (!(ok = wait(bar(kBarKFull0 + s), par))) break;
-                const int j = ctrl.list[kbeg + k] & 0x1FFF;
-                const int row = j * kTileRows + r;
-                uint8_t* kt = smem + L::kK0 + s * L::kKStage;
-                if (row < p.key_rows)
-                    rope_key_row<D>(kt, kt + L::kTileBytes, r, p.rope + (size_t)key_pos(p.w, row) * (D / 2));
-                else
-                    zero_key_row<D>(kt, kt + L::kTileBytes, r);
-                fence_proxy_async_smem();
-                mbar_arrive(bar(kBarKRot0 + s));
-                if (!(ok = wait(bar(kBarVFull0 + s), par))) break;
-                v_row_to_f16<D>(smem + L::kV0 + s * L::kTileBytes, r);
-                fence_proxy_async_smem();
-                mbar_arrive(bar(kBarVConv0 + s));
-            }
+            const int t = t0 + r / p.G;
+            const int h = kvh * p.G + r % p.G;
+            // Rows past the last token rotate a valid row (token t0) and are never stored.
+            const int tt = t < t_end ? t : t0;
+            const int qp = query_pos(p.w, p.q_mode, tt);
+            rope_query_row<D>(Q + ((size_t)tt * p.H + h) * D, p.rope + (size_t)qp * (D / 2), p.q_scale,
+                              tmem + kColQ + lane_off, tmem + kColQ + D / 2 + lane_off);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(kBarQReady));
         }
     }
 
@@ -617,8 +561,8 @@ __global__ void wait_probe_kernel(unsigned* err, unsigned long long limit_ns) {
 }
 
 template <int D>
-cudaError_t launch_d(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tk, const CUtensorMap& tv,
-                     cudaStream_t stream) {
+cudaError_t launch_d(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tkh, const CUtensorMap& tkl,
+                     const CUtensorMap& tv16, cudaStream_t stream) {
     const size_t smem = stream_attn_smem_bytes(D);
     static bool attr = false;
     if (!attr) {
@@ -628,7 +572,7 @@ cudaError_t launch_d(const AttnParams& p, const uint16_t* Q, const CUtensorMap& 
         attr = true;
     }
     const unsigned grid = unsigned(p.Hkv * p.q_tiles * p.splits);
-    stream_attn_kernel<D><<<grid, kThreads, smem, stream>>>(p, Q, tk, tv);
+    stream_attn_kernel<D><<<grid, kThreads, smem, stream>>>(p, Q, tkh, tkl, tv16);
     return cudaGetLastError();
 }
 
@@ -640,9 +584,9 @@ size_t stream_attn_smem_bytes(int d) {
     return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
-cudaError_t launch_stream_attn(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tk, const CUtensorMap& tv,
-                               cudaStream_t stream) {
-    return p.d == 128 ? launch_d<128>(p, Q, tk, tv, stream) : launch_d<64>(p, Q, tk, tv, stream);
+cudaError_t launch_stream_attn(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tkh,
+                               const CUtensorMap& tkl, const CUtensorMap& tv16, cudaStream_t stream) {
+    return p.d == 128 ? launch_d<128>(p, Q, tkh, tkl, tv16, stream) : launch_d<64>(p, Q, tkh, tkl, tv16, stream);
 }
 
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream) {
