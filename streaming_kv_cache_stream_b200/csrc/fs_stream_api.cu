@@ -46,7 +46,9 @@ struct fs_stream {
     int part_rows_cap = 0;  // rows of 128 query rows x d fp32 the split scratch holds
     void* stage = nullptr;  // host-path staging: K, V, Q, out
     size_t stage_bytes = 0;
-    CUtensorMap tmap_k, tmap_v, tmap_kh, tmap_kl, tmap_v16;
+    CUtensorMap tmap_k, tmap_v;                 // bf16 cache, full 128-row tiles (rope loads)
+    CUtensorMap tmap_kh, tmap_kl, tmap_v16;     // fp16 operands, full tiles (rope stores)
+    CUtensorMap tmap_kh2, tmap_kl2, tmap_v16h;  // fp16 operands, one CTA's half tile (attention loads)
     unsigned long long wait_limit_ns = 2000000000ull;
     long long cache_bytes = 0;
     long long launches = 0;
@@ -87,18 +89,20 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// 3-D 16-bit tensor map, 128-byte swizzle, box {64, b1, b2}, out-of-range reads as zero.
+// 3-D 16-bit tensor map, box {b0, b1, b2}, out-of-range reads as zero; 128-byte
+// swizzle unless told otherwise.
 int make_map(fs_stream_t s, CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
              uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b1, uint32_t b2,
-             CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+             CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint32_t b0 = 64,
+             CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto enc = get_encode();
     if (!enc) return fail(s, FS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
     cuuint64_t dims[3] = {d0, d1, d2};
     cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-    cuuint32_t box[3] = {64, b1, b2};
+    cuuint32_t box[3] = {b0, b1, b2};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(s, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
     return FS_OK;
@@ -163,14 +167,18 @@ int do_insert(fs_stream_t s, const void* K, const void* V, int n_tokens, int mod
     return FS_OK;
 }
 
-// Splits of the key range per (kv head, query tile) so that small query sets
-// still fill the SMs; capped by the scratch and by the number of key tiles.
-int choose_splits(const fs_stream* s, int items, int key_rows) {
-    if (items >= s->num_sms) return 1;
+// Splits of the key range per (kv head, pair of query tiles) so that small
+// query sets still fill the SMs (a pair occupies two); capped by the scratch
+// (one partial per query tile and split) and by the number of key tiles.
+int choose_splits(const fs_stream* s, int q_tiles, int key_rows) {
+    const int pairs = ((q_tiles + 1) / 2) * s->Hkv;
+    const int slots = s->num_sms / 2;
+    if (pairs >= slots) return 1;
     const int ktiles = (key_rows + fs::kTileRows - 1) / fs::kTileRows;
-    int sp = (s->num_sms + items - 1) / items;
+    int sp = (slots + pairs - 1) / pairs;
     if (sp > ktiles / 2) sp = ktiles / 2;
-    if (sp > s->part_rows_cap / items) sp = s->part_rows_cap / items;
+    const int tiles_padded = 2 * pairs;
+    if (sp > s->part_rows_cap / tiles_padded) sp = s->part_rows_cap / tiles_padded;
     return sp < 1 ? 1 : sp;
 }
 
@@ -186,7 +194,7 @@ int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key
     p.nq = nq;
     p.q_mode = mode;
     p.q_tiles = q_tiles;
-    p.splits = choose_splits(s, s->Hkv * q_tiles, key_rows);
+    p.splits = choose_splits(s, q_tiles, key_rows);
     p.q_scale = float(1.4426950408889634 / std::sqrt(double(s->d)));
     p.rope = s->rope;
     p.rope_rows = s->rope_rows;
@@ -205,7 +213,7 @@ int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key
     rp.wait_limit_ns = s->wait_limit_ns;
     FS_CUDA(s, fs::launch_kv_stream_rope(rp, s->tmap_k, s->tmap_v, s->tmap_kh, s->tmap_kl, s->tmap_v16, s->stream));
     s->launches += 1;
-    FS_CUDA(s, fs::launch_stream_attn(p, static_cast<const uint16_t*>(Q), s->tmap_kh, s->tmap_kl, s->tmap_v16,
+    FS_CUDA(s, fs::launch_stream_attn(p, static_cast<const uint16_t*>(Q), s->tmap_kh2, s->tmap_kl2, s->tmap_v16h,
                                       s->stream));
     s->launches += 1;
     if (p.splits > 1) {
@@ -308,6 +316,14 @@ int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame,
                            fs::kTileRows, 1, f16);
     if (!rc) rc = make_map(nullptr, &s->tmap_v16, s->V16, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
                            fs::kTileRows, 1, f16);
+    // Pair loads: 64 key rows of K hi / lo; all 128 key rows of d/2 V columns.
+    if (!rc) rc = make_map(nullptr, &s->tmap_kh2, s->Kh, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
+                           fs::kTileRows / 2, 1, f16);
+    if (!rc) rc = make_map(nullptr, &s->tmap_kl2, s->Kl, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
+                           fs::kTileRows / 2, 1, f16);
+    if (!rc) rc = make_map(nullptr, &s->tmap_v16h, s->V16, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
+                           fs::kTileRows, 1, f16, uint32_t(d / 2),
+                           d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
     if (rc) return bail(rc);
     *out = s;
     return FS_OK;

@@ -194,6 +194,7 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // ------------------------------------------------------------- descriptors
 
 // Shared-memory matrix descriptor for tcgen05.mma (sm_100 format):
+// (64-byte swizzle, MN-major: 32-element MN atoms, 8-row K groups 512 bytes apart.)
 //   bits  0-13 start address >> 4, 16-29 leading-dim byte offset >> 4,
 //   bits 32-45 stride-dim byte offset >> 4, bits 46-47 version (1),
 //   bits 49-51 base offset (0: atoms 1024-byte aligned), bits 61-63 layout
@@ -201,14 +202,19 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // K-major, 128B swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart (SBO);
 // LBO unused (1). MN-major, 128B swizzle: 64-element MN atoms `lbo` bytes
 // apart, 8-row K groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+// Layout codes (bits 61-63): 2 = 128-byte swizzle, 4 = 64-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
     uint64_t d = 0;
     d |= uint64_t((saddr >> 4) & 0x3FFF);
     d |= uint64_t((lbo_bytes >> 4) & 0x3FFF) << 16;
     d |= uint64_t((sbo_bytes >> 4) & 0x3FFF) << 32;
     d |= uint64_t(1) << 46;
-    d |= uint64_t(2) << 61;
+    d |= uint64_t(layout & 7) << 61;
     return d;
+}
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return smem_desc(saddr, lbo_bytes, sbo_bytes, 2);
 }
 
 // Instruction descriptor, kind::f16: c_format F32 (bit 4), a/b formats at bits 7/10
@@ -217,6 +223,92 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_bf16, bool b_bf16, bool a_mn, bool b_mn) {
     return (1u << 4) | (uint32_t(a_bf16) << 7) | (uint32_t(b_bf16) << 10) | (uint32_t(a_mn) << 15) |
            (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// ------------------------------------------------ CTA pairs (cta_group::2)
+// A cluster of two CTAs on two SMs shares one MMA of M = 256: each CTA holds
+// its 128 rows of A and D and half of B's N columns. The even CTA (rank 0)
+// issues the MMAs; completion is multicast to both CTAs' mbarriers.
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory offset in the cluster CTA of rank `rank`.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (any CTA of the
+// cluster), default (.release.cta) semantics: the data handed over is in TMEM
+// and is ordered by tcgen05.fence::before_thread_sync, so no cluster-scope
+// release of generic memory is needed (measured 0.6 us per arrive).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Pair TMA load: data lands in this CTA's shared memory, the byte count is
+// credited to the mbarrier at `bar_cluster` (the leader's).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                                 uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Pair MMA, A from TMEM (each CTA's own 128 rows), B from shared memory (each
+// CTA's half of N at the same offset), D in each CTA's TMEM.
+__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Pair MMA with A from shared memory (each CTA's own 128 rows at the same offset).
+__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on the mbarrier at this offset in both CTAs of the pair when the
+// pair MMAs issued so far by this thread are done.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    const uint16_t both = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            bar),
+        "h"(both)
+        : "memory");
 }
 
 // ----------------------------------------------------------- small numerics
@@ -244,6 +336,11 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
 __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {

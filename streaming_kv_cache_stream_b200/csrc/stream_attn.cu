@@ -7,26 +7,34 @@
 // new-frame and text queries attend under the streaming mask "query p sees key
 // q iff pos(q) <= pos(p)".
 //
-// One CTA = one (kv head, 128-row query tile[, key split]). A query tile packs
-// 128/G tokens x the G query heads that share the kv head, so every key tile
-// is loaded once for all G heads (GQA). The keys were rotated once for this
-// step by kv_stream_rope (RoPE in shared memory at their shifted positions,
-// written as fp16 hi + lo, V as fp16); this kernel rotates its query rows.
-// Warp roles, 12 warps:
-//   warp 0      TMA producer: K hi + K lo tile and V tile, two stages each;
-//   warp 1      TMEM allocator and tcgen05.mma issuer (one thread);
-//   warps 4-7   softmax: one query row per thread; S read from TMEM, streaming
-//               mask, online softmax in fp32 with exp2, P written back into
-//               TMEM over S, lazy rescale of O in TMEM, epilogue;
-//   warps 8-11  RoPE of the query rows at their window positions, written into
-//               TMEM as the A operand (fp16 hi + lo), once per CTA.
-// Pipeline per key tile j (S double-buffered in TMEM):
-//   TMA K_j, V_j -> MMA S_j = Q K_j^T -> softmax(S_j) -> P_j -> MMA O += P_j V_j;
-//   QK_{j+1} is issued before PV_j, so the tensor core works on the next tile
-//   while the softmax warps run.
+// Work unit: a pair of CTAs on two SMs (a cluster of 2, tcgen05 cta_group::2)
+// takes two 128-row query tiles of one kv head and runs M = 256 MMAs: each
+// CTA holds its own 128 query rows (Q in shared memory, S and O in its TMEM)
+// and half of every key tile (64 of the 128 keys) and V tile (D/2 of the
+// columns), so a key tile crosses the memory system once per pair. A query
+// tile packs 128/G tokens x the G query heads of one kv group (GQA). The keys
+// were rotated for this step by kv_stream_rope (at their shifted positions, as
+// fp16 hi + lo; V as fp16); this kernel rotates its query rows.
+//
+// Warp roles per CTA (12 warps):
+//   warp 0      TMA producer: this CTA's halves of K hi/lo and V, 3 stages;
+//   warp 1      TMEM allocation; in the even CTA, the single MMA issuer;
+//   warps 4-7   softmax of the even key tiles (S buffer 0, O accumulator 0);
+//   warps 8-11  RoPE of the query rows into shared memory, then softmax of the
+//               odd key tiles (S buffer 1, O accumulator 1).
+// The two softmax warpgroups each keep their own running max and sum over
+// their half of the key tiles and their own O; the epilogue merges the two
+// (as a split of the key range would be merged). So they never wait for each
+// other, each has two MMA periods per tile, and the lazy O rescale never
+// stalls: QK of tile k already waits for PV of tile k-2, the last write to
+// the same O.
+// Pipeline: TMA K_j,V_j -> MMA S_j = Q K_j^T (into S_{j%2}) -> softmax ->
+// P_j (fp16, over S in TMEM) -> MMA O_{j%2} += P_j V_j; QK_{j+1} is issued
+// before PV_j.
 // Key tiles are walked in physical ring order; positions come from key_pos(),
-// so the ring never moves. Tiles whose every key is after the tile's last
-// query are skipped; tiles that are entirely visible skip the elementwise mask.
+// so the ring never moves. Tiles whose every key is after the pair's last
+// query are skipped; tiles entirely visible to the pair skip the elementwise
+// mask.
 //
 // Precision. Rotation happens in fp32 from the bf16 inputs and a table of
 // fp32 cos/sin evaluated in double. The rotated Q (pre-scaled by log2(e)/sqrt(d))
@@ -37,9 +45,9 @@
 // the scores to ~2^-22 relative. P is fp16 (V is fp16 to match), O
 // accumulates in fp32, and the output is stored in fp32.
 //
-// Shared-memory tiles use the 128-byte swizzle that TMA writes and tcgen05
-// reads: rows of 128 bytes, 16-byte chunk c of row r at chunk position
-// c ^ (r & 7); head dims 64..127 live in a second 16 KB region.
+// Shared-memory tiles use the swizzled layouts TMA writes and tcgen05 reads:
+// 128-byte rows with 16-byte chunk c of row r at chunk position c ^ (r & 7)
+// (head dims 64..127 in a second region), or 64-byte rows for V at D = 64.
 #include <cfloat>
 #include <climits>
 
@@ -50,24 +58,37 @@ namespace fs {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kRegion = 16384;           // 128 rows x 128 bytes
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;          // O: 256 .. 256+D
-constexpr uint32_t kColQ = 384;          // Q hi: 384 .. 384+D/2, Q lo: 384+D/2 .. 384+D
-constexpr float kRescaleLog2 = 8.0f;     // rescale O only when the max grows by > 2^8
+constexpr uint32_t kColO0 = 256;         // O accumulators: 256 .. 256+D and 384 .. 384+D
+constexpr uint32_t kColO1 = 384;
+// Rescale O only when the running max grows by more than 2^14: P = 2^(s - m)
+// then stays below 2^14 (fp16 holds up to 65504), so most tiles skip it.
+constexpr float kRescaleLog2 = 14.0f;
+constexpr int kStages = 3;               // K and V operand stages per CTA
 
 __device__ __forceinline__ constexpr uint32_t col_s(int s) { return s ? 128u : 0u; }
+__device__ __forceinline__ constexpr uint32_t col_o(int s) { return s ? kColO1 : kColO0; }
 
 enum : int {
-    kBarQReady = 0, kBarKFull0, kBarKFull1, kBarKEmpty0, kBarKEmpty1, kBarVFull0, kBarVFull1,
-    kBarVEmpty0, kBarVEmpty1, kBarSFull0, kBarSFull1, kBarPFull0, kBarPFull1, kBarSFree0, kBarSFree1,
-    kBarOFull, kBarMmaDone, kNumBars
+    kBarQReady = 0,
+    kBarKFull0 = 1,
+    kBarKEmpty0 = kBarKFull0 + kStages,
+    kBarVFull0 = kBarKEmpty0 + kStages,
+    kBarVEmpty0 = kBarVFull0 + kStages,
+    kBarSFull0 = kBarVEmpty0 + kStages,
+    kBarPFull0 = kBarSFull0 + 2,
+    kBarSFree0 = kBarPFull0 + 2,
+    kBarOFull0 = kBarSFree0 + 2,
+    kBarMmaDone = kBarOFull0 + 2,
+    kNumBars
 };
 
 constexpr uint8_t kSkip = 0, kFull = 1, kPartial = 2;
 
 struct Ctrl {
-    alignas(16) int kpos[2][kTileRows];
+    alignas(16) int kpos[2][2][kTileRows];  // [warpgroup][buffer][key]: positions of a masked tile's keys
+    float red_m[2][kTileRows];              // [warpgroup][row]: final running max (epilogue merge)
+    float red_l[2][kTileRows];              // [warpgroup][row]: final running sum
     uint64_t bars[kNumBars];
     uint32_t tmem_base;
     int nvis;
@@ -75,13 +96,25 @@ struct Ctrl {
     uint8_t cls[kMaxKeyTiles];
 };
 
+// Per-CTA shared memory: the CTA's 128 query rows as fp16 hi and lo (128-byte
+// swizzle, head dims 64..127 in a second region), then 3 stages, each with
+// this CTA's half of a key tile (64 of the 128 keys, K hi then K lo) and its
+// half of the V tile (all 128 keys, D/2 of the columns; 128-byte swizzle at
+// D = 128, 64-byte swizzle at D = 64).
 template <int D>
 struct Layout {
-    static constexpr int kTileBytes = kTileRows * D * 2;   // one [128 x D] 16-bit tile
-    static constexpr int kK0 = 0;                          // K stage s: hi tile then lo tile
-    static constexpr int kKStage = 2 * kTileBytes;
-    static constexpr int kV0 = 2 * kKStage;                // V stage s
-    static constexpr int kCtrl = kV0 + 2 * kTileBytes;
+    static constexpr int kQRegion = 128 * 128;               // 128 rows x 128 bytes
+    static constexpr int kQHalf = 128 * D * 2;               // one of Q hi / Q lo
+    static constexpr int kKRegion = 64 * 128;                // 64 key rows x 128 bytes
+    static constexpr int kKHalf = 64 * D * 2;                // one of K hi / K lo
+    static constexpr int kKStage = 2 * kKHalf;
+    static constexpr int kVRow = D;                          // bytes per key row of the V half (D/2 x 2)
+    static constexpr int kVStage = kTileRows * kVRow;
+    static constexpr uint32_t kVLayout = D == 128 ? 2u : 4u; // 128- or 64-byte swizzle
+    static constexpr int kQ = 0;
+    static constexpr int kK0 = 2 * kQHalf;
+    static constexpr int kV0 = kK0 + kStages * kKStage;
+    static constexpr int kCtrl = kV0 + kStages * kVStage;
     static constexpr int kBytes = kCtrl + int(sizeof(Ctrl));
 };
 
@@ -106,89 +139,86 @@ __device__ __forceinline__ void key_bounds(const WindowShape& w, int r0, int r1,
     }
 }
 
-// fp32 -> fp16 hi + fp16 lo (lo = the rounding residual), packed in pairs.
+// fp32 pair -> fp16 hi pair + fp16 lo pair (lo = the rounding residual of hi).
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
     hi = pack_f16x2(a, b);
-    const __half2 h = *reinterpret_cast<const __half2*>(&hi);
-    const float2 hf = __half22float2(h);
+    const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hi));
     lo = pack_f16x2(a - hf.x, b - hf.y);
 }
 
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-                 : "memory");
-}
-
-// Rotates this thread's query row (loaded from global memory, pre-RoPE bf16),
-// scales it by q_scale, and writes fp16 hi / lo parts into TMEM (K-major A
-// operand: element i of the row at column i/2, two fp16 per column).
+// Rotates one query row (pre-RoPE bf16 in global memory) by the angles in
+// `cs`, scales it by `scale`, and writes it as fp16 hi / lo into row `row` of
+// the swizzled Q tiles `qhi` / `qlo` (the K-major A operand of the QK MMA).
+// Pair (i, i + D/2): for D = 128 chunk c of region 0 pairs with chunk c of
+// region 1; for D = 64 chunk c pairs with chunk c + 4.
 template <int D>
 __device__ __forceinline__ void rope_query_row(const uint16_t* __restrict__ qrow, const float2* __restrict__ cs,
-                                               float scale, uint32_t t_hi, uint32_t t_lo) {
-    constexpr int kHalf = D / 2;
-    constexpr int kM = kHalf / 16;  // 16-element blocks per half
+                                               float scale, uint8_t* qhi, uint8_t* qlo, int row) {
+    constexpr int kPairs = D / 16;
+    const int sw = row & 7;
 #pragma unroll
-    for (int m0 = 0; m0 < kM; m0 += 2) {
-        // Issue every load of two blocks before any arithmetic: one round trip per pair.
-        uint4 qa[2][2], qb[2][2];
-        float4 tt[2][8];
+    for (int c0 = 0; c0 < kPairs; c0 += 2) {
+        // Two chunk pairs per round: every load is issued before the arithmetic.
+        uint4 a[2], b[2];
+        float4 t[2][4];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const int m = m0 + u;
-            if (m < kM) {
-                const uint4* pa = reinterpret_cast<const uint4*>(qrow + 16 * m);
-                const uint4* pb = reinterpret_cast<const uint4*>(qrow + kHalf + 16 * m);
-                qa[u][0] = __ldg(pa);
-                qa[u][1] = __ldg(pa + 1);
-                qb[u][0] = __ldg(pb);
-                qb[u][1] = __ldg(pb + 1);
-                const float4* t4 = reinterpret_cast<const float4*>(cs + 16 * m);
+            const int c = c0 + u;
+            a[u] = __ldg(reinterpret_cast<const uint4*>(qrow + 8 * c));
+            b[u] = __ldg(reinterpret_cast<const uint4*>(qrow + D / 2 + 8 * c));
+            const float4* t4 = reinterpret_cast<const float4*>(cs + 8 * c);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) tt[u][q] = __ldg(t4 + q);
-            }
+            for (int q = 0; q < 4; ++q) t[u][q] = __ldg(t4 + q);
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const int m = m0 + u;
-            if (m >= kM) break;
-            const uint32_t aw[8] = {qa[u][0].x, qa[u][0].y, qa[u][0].z, qa[u][0].w,
-                                    qa[u][1].x, qa[u][1].y, qa[u][1].z, qa[u][1].w};
-            const uint32_t bw[8] = {qb[u][0].x, qb[u][0].y, qb[u][0].z, qb[u][0].w,
-                                    qb[u][1].x, qb[u][1].y, qb[u][1].z, qb[u][1].w};
-            uint32_t ah[8], al[8], bh[8], bl[8];
+            const int c = c0 + u;
+            const int oa = row * 128 + ((c ^ sw) << 4);
+            const int ob = D == 128 ? oa + Layout<D>::kQRegion : row * 128 + (((c + 4) ^ sw) << 4);
+            const uint32_t aw[4] = {a[u].x, a[u].y, a[u].z, a[u].w};
+            const uint32_t bw[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
+            uint32_t ah[4], al[4], bh[4], bl[4];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 t = tt[u][q];  // (cos, sin) of elements 16m + 2q, 16m + 2q + 1
+            for (int q = 0; q < 4; ++q) {
+                const float4 tq = t[u][q];  // (cos, sin) of elements 8c + 2q and 8c + 2q + 1
                 const float x0 = bf16lo(aw[q]), x1 = bf16hi(aw[q]);
                 const float y0 = bf16lo(bw[q]), y1 = bf16hi(bw[q]);
-                split2((x0 * t.x - y0 * t.y) * scale, (x1 * t.z - y1 * t.w) * scale, ah[q], al[q]);
-                split2((y0 * t.x + x0 * t.y) * scale, (y1 * t.z + x1 * t.w) * scale, bh[q], bl[q]);
+                split2((x0 * tq.x - y0 * tq.y) * scale, (x1 * tq.z - y1 * tq.w) * scale, ah[q], al[q]);
+                split2((y0 * tq.x + x0 * tq.y) * scale, (y1 * tq.z + x1 * tq.w) * scale, bh[q], bl[q]);
             }
-            tmem_st8(t_hi + 8 * m, ah);
-            tmem_st8(t_hi + kHalf / 2 + 8 * m, bh);
-            tmem_st8(t_lo + 8 * m, al);
-            tmem_st8(t_lo + kHalf / 2 + 8 * m, bl);
+            *reinterpret_cast<uint4*>(qhi + oa) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
+            *reinterpret_cast<uint4*>(qhi + ob) = make_uint4(bh[0], bh[1], bh[2], bh[3]);
+            *reinterpret_cast<uint4*>(qlo + oa) = make_uint4(al[0], al[1], al[2], al[3]);
+            *reinterpret_cast<uint4*>(qlo + ob) = make_uint4(bl[0], bl[1], bl[2], bl[3]);
         }
     }
 }
 
-__device__ __forceinline__ bool vote_all_ok_wg(bool ok) {
-    // Uniform decision over the 128 softmax threads (named barrier 1).
+// Uniform decision over `threads` threads at named barrier `id`: true iff all pass `ok`.
+__device__ __forceinline__ bool vote_all_ok(uint32_t id, uint32_t threads, bool ok) {
     uint32_t res;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.red.and.pred q, 1, 128, p;\n\t"
+        "setp.ne.u32 p, %3, 0;\n\t"
+        "barrier.red.and.pred q, %1, %2, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(res)
-        : "r"(uint32_t(ok))
+        : "r"(id), "r"(threads), "r"(uint32_t(ok))
         : "memory");
     return res != 0;
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     stream_attn_kernel(const __grid_constant__ AttnParams p, const uint16_t* __restrict__ Q,
                        const __grid_constant__ CUtensorMap tkh, const __grid_constant__ CUtensorMap tkl,
                        const __grid_constant__ CUtensorMap tv16) {
@@ -199,43 +229,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
+    const uint32_t rank = cluster_rank();  // 0: leader (issues the pair's MMAs), 1: peer
+    const bool leader = rank == 0;
 
-    // ---- work item: heavy query tiles (later tokens see more keys) first
-    const int split = blockIdx.x % p.splits;
-    const int item = blockIdx.x / p.splits;
-    const int qt = p.q_tiles - 1 - item / p.Hkv;
+    // ---- work item: a pair of query tiles (2 pq, 2 pq + 1) of one kv head; heavy
+    // pairs (later tokens see more keys) first.
+    const int pair_id = blockIdx.x >> 1;
+    const int split = pair_id % p.splits;
+    const int item = pair_id / p.splits;
+    const int q_pairs = (p.q_tiles + 1) >> 1;
+    const int pq = q_pairs - 1 - item / p.Hkv;
     const int kvh = item % p.Hkv;
+    const int qt = 2 * pq + int(rank);
+    const bool tile_valid = qt < p.q_tiles;
     const int item_id = qt * p.Hkv + kvh;
     const int tok_per_tile = kTileRows / p.G;
     const int t0 = qt * tok_per_tile;
     const int t_end = min(t0 + tok_per_tile, p.nq);
-    const int qmin = query_pos(p.w, p.q_mode, t0);
-    const int qmax = query_pos(p.w, p.q_mode, t_end - 1);
+    // Query-position range of the pair (the union of its valid tiles; positions grow with tokens).
+    const int pair_t0 = 2 * pq * tok_per_tile;
+    const int pair_t1 = min(pair_t0 + 2 * tok_per_tile, p.nq);
+    const int qmin = query_pos(p.w, p.q_mode, pair_t0);
+    const int qmax = query_pos(p.w, p.q_mode, pair_t1 - 1);
     const BoundedWait wait{p.err, p.wait_limit_ns, kErrTimeout};
 
     auto bar = [&](int i) { return smem_u32(&ctrl.bars[i]); };
+    auto lbar = [&](int i) { return map_to_rank(smem_u32(&ctrl.bars[i]), 0); };  // the leader's copy
 
     if (tid == 0) {
-        mbar_init(bar(kBarQReady), 128);
-        for (int s = 0; s < 2; ++s) {
+        mbar_init(bar(kBarQReady), 8);  // one arrival per RoPE warp of both CTAs
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(kBarKFull0 + s), 1);
             mbar_init(bar(kBarKEmpty0 + s), 1);
             mbar_init(bar(kBarVFull0 + s), 1);
             mbar_init(bar(kBarVEmpty0 + s), 1);
-            mbar_init(bar(kBarSFull0 + s), 1);
-            mbar_init(bar(kBarPFull0 + s), 128);
-            mbar_init(bar(kBarSFree0 + s), 1);
         }
-        mbar_init(bar(kBarOFull), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(kBarSFull0 + s), 1);
+            mbar_init(bar(kBarPFull0 + s), 8);  // one arrival per softmax warp of that buffer, both CTAs
+            mbar_init(bar(kBarSFree0 + s), 1);
+            mbar_init(bar(kBarOFull0 + s), 1);
+        }
         mbar_init(bar(kBarMmaDone), 1);
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&ctrl.tmem_base), kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32(&ctrl.tmem_base), kTmemCols);
+        tmem_relinquish_pair();
     }
 
-    // ---- classify key tiles against this query tile, then list the visible ones
+    // ---- classify key tiles against the pair's query range, then list the visible ones
     const int n_ktiles = (p.key_rows + kTileRows - 1) / kTileRows;
     for (int j = tid; j < n_ktiles; j += kThreads) {
         const int r0 = j * kTileRows;
@@ -264,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or commit
     tc_fence_after();
     const uint32_t tmem = ctrl.tmem_base;
     const int nvis = ctrl.nvis;
@@ -272,122 +316,145 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nt = kend - kbeg;
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;  // TMEM lanes of this warp
 
-    // Register split, one setmaxnreg per warpgroup at the head of its region: the
-    // softmax warpgroup holds a 128-column S row per thread.
-    // 128 x (80 + 232 + 192) <= 384 x 168, the registers allocated at launch.
+    // Register split, one setmaxnreg per warpgroup at the head of its region:
+    // 128 x (80 + 208 + 208) <= 384 x 168, the registers allocated at launch.
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
         if (warp == 0) {
-            // ============================================= TMA producer
+            // ============================================= TMA producer (both CTAs)
+            // Each CTA loads its half of every operand tile: keys [64 r, 64 r + 64)
+            // of K hi/lo, columns [D/2 r, D/2 r + D/2) of V; the leader's full
+            // barriers count the bytes of both CTAs.
             if (lane == 0 && nt > 0) {
                 tma_prefetch_desc(&tkh);
                 tma_prefetch_desc(&tkl);
                 tma_prefetch_desc(&tv16);
                 for (int k = 0; k < nt; ++k) {
-                    const int s = k & 1;
-                    const uint32_t par = ((k >> 1) & 1) ^ 1;
+                    const int s = k % kStages;
+                    const uint32_t par = ((k / kStages) & 1) ^ 1;
                     const int j = ctrl.list[kbeg + k] & 0x1FFF;
                     if (!wait(bar(kBarKEmpty0 + s), par)) break;
-                    mbar_arrive_expect_tx(bar(kBarKFull0 + s), 2 * L::kTileBytes);
+                    if (leader) mbar_arrive_expect_tx(bar(kBarKFull0 + s), 2 * L::kKStage);
                     const uint32_t kd = smem_u32(smem + L::kK0 + s * L::kKStage);
 #pragma unroll
                     for (int r = 0; r < D / 64; ++r) {
-                        tma_load_3d(kd + r * kRegion, &tkh, r * 64, j * kTileRows, kvh, bar(kBarKFull0 + s));
-                        tma_load_3d(kd + L::kTileBytes + r * kRegion, &tkl, r * 64, j * kTileRows, kvh,
-                                    bar(kBarKFull0 + s));
+                        tma_load_3d_pair(kd + r * L::kKRegion, &tkh, r * 64, j * kTileRows + 64 * int(rank), kvh,
+                                         lbar(kBarKFull0 + s));
+                        tma_load_3d_pair(kd + L::kKHalf + r * L::kKRegion, &tkl, r * 64,
+                                         j * kTileRows + 64 * int(rank), kvh, lbar(kBarKFull0 + s));
                     }
                     if (!wait(bar(kBarVEmpty0 + s), par)) break;
-                    mbar_arrive_expect_tx(bar(kBarVFull0 + s), L::kTileBytes);
-                    const uint32_t vd = smem_u32(smem + L::kV0 + s * L::kTileBytes);
-#pragma unroll
-                    for (int r = 0; r < D / 64; ++r)
-                        tma_load_3d(vd + r * kRegion, &tv16, r * 64, j * kTileRows, kvh, bar(kBarVFull0 + s));
+                    if (leader) mbar_arrive_expect_tx(bar(kBarVFull0 + s), 2 * L::kVStage);
+                    tma_load_3d_pair(smem_u32(smem + L::kV0 + s * L::kVStage), &tv16, (D / 2) * int(rank),
+                                     j * kTileRows, kvh, lbar(kBarVFull0 + s));
                 }
             }
         } else if (warp == 1) {
-            // ============================================= MMA issuer
-            if (lane == 0 && nt > 0) {
-                constexpr uint32_t idesc_qk = idesc_f16(128, 128, false, false, false, false);
-                constexpr uint32_t idesc_pv = idesc_f16(128, D, false, false, false, true);
-                const uint32_t q_hi = tmem + kColQ, q_lo = tmem + kColQ + D / 2;
+            // ============================================= MMA issuer (leader CTA only)
+            if (leader && lane == 0 && nt > 0) {
+                constexpr uint32_t idesc_qk = idesc_f16(256, 128, false, false, false, false);
+                constexpr uint32_t idesc_pv = idesc_f16(256, D, false, false, false, true);
+                // Descriptors are formed once; a K step advances the start-address
+                // field (bits 0-13, in 16-byte units) by the step's offset.
+                const uint64_t dqh = sw128_desc(smem_u32(smem + L::kQ), 16, 1024);
+                const uint64_t dql = dqh + (L::kQHalf >> 4);
+                const uint64_t dk0 = sw128_desc(smem_u32(smem + L::kK0), 16, 1024);
+                const uint64_t dv0 = smem_desc(smem_u32(smem + L::kV0), L::kVStage, 8 * L::kVRow, L::kVLayout);
                 bool ok = wait(bar(kBarQReady), 0);
                 for (int k = 0; ok && k <= nt; ++k) {
                     if (k < nt) {
-                        const int s = k & 1;
-                        if (!(ok = wait(bar(kBarKFull0 + s), (k >> 1) & 1))) break;
-                        if (k >= 2 && !(ok = wait(bar(kBarSFree0 + s), ((k - 2) >> 1) & 1))) break;
+                        const int s = k % kStages;
+                        const int sb = k & 1;
+                        if (!(ok = wait(bar(kBarKFull0 + s), (k / kStages) & 1))) break;
+                        if (k >= 2 && !(ok = wait(bar(kBarSFree0 + sb), ((k - 2) >> 1) & 1))) break;
                         tc_fence_after();
-                        const uint32_t kh = smem_u32(smem + L::kK0 + s * L::kKStage);
-                        const uint32_t kl = kh + L::kTileBytes;
-                        const uint32_t d_s = tmem + col_s(s);
+                        const uint64_t dkh = dk0 + uint32_t((s * L::kKStage) >> 4);
+                        const uint64_t dkl = dkh + (L::kKHalf >> 4);
+                        const uint32_t d_s = tmem + col_s(sb);
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-                            const uint64_t dh = sw128_desc(kh + off, 16, 1024);
-                            const uint64_t dl = sw128_desc(kl + off, 16, 1024);
-                            mma_ts(d_s, q_hi + 8 * kk, dh, idesc_qk, kk > 0);
-                            mma_ts(d_s, q_hi + 8 * kk, dl, idesc_qk, 1);
-                            mma_ts(d_s, q_lo + 8 * kk, dh, idesc_qk, 1);
+                            const uint32_t qo = ((kk >> 2) * L::kQRegion + (kk & 3) * 32) >> 4;
+                            const uint32_t ko = ((kk >> 2) * L::kKRegion + (kk & 3) * 32) >> 4;
+                            mma_ss_pair(d_s, dqh + qo, dkh + ko, idesc_qk, kk > 0);
+                            mma_ss_pair(d_s, dqh + qo, dkl + ko, idesc_qk, 1);
+                            mma_ss_pair(d_s, dql + qo, dkh + ko, idesc_qk, 1);
                         }
-                        tc_commit(bar(kBarSFull0 + s));
-                        tc_commit(bar(kBarKEmpty0 + s));
+                        tc_commit_pair(bar(kBarSFull0 + sb));
+                        tc_commit_pair(bar(kBarKEmpty0 + s));
                     }
                     if (k >= 1) {
                         const int kp = k - 1;
-                        const int s = kp & 1;
-                        const uint32_t par = (kp >> 1) & 1;
-                        if (!(ok = wait(bar(kBarPFull0 + s), par))) break;
-                        if (!(ok = wait(bar(kBarVFull0 + s), par))) break;
+                        const int s = kp % kStages;
+                        const int sb = kp & 1;
+                        if (!(ok = wait(bar(kBarPFull0 + sb), (kp >> 1) & 1))) break;
+                        if (!(ok = wait(bar(kBarVFull0 + s), (kp / kStages) & 1))) break;
                         tc_fence_after();
-                        const uint32_t vs = smem_u32(smem + L::kV0 + s * L::kTileBytes);
+                        const uint64_t dv = dv0 + uint32_t((s * L::kVStage) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < kTileRows / 16; ++kk)
-                            mma_ts(tmem + kColO, tmem + col_s(s) + kk * 8, sw128_desc(vs + kk * 2048, kRegion, 1024),
-                                   idesc_pv, (kp > 0 || kk > 0));
-                        tc_commit(bar(kBarVEmpty0 + s));
-                        tc_commit(bar(kBarSFree0 + s));
-                        tc_commit(bar(kBarOFull));
+                            mma_ts_pair(tmem + col_o(sb), tmem + col_s(sb) + kk * 8, dv + ((kk * 16 * L::kVRow) >> 4),
+                                        idesc_pv, (kp >= 2 || kk > 0));
+                        tc_commit_pair(bar(kBarVEmpty0 + s));
+                        tc_commit_pair(bar(kBarSFree0 + sb));
+                        tc_commit_pair(bar(kBarOFull0 + sb));
                     }
                 }
                 // Drain: every MMA issued above completes before TMEM is released.
-                tc_commit(bar(kBarMmaDone));
+                tc_commit_pair(bar(kBarMmaDone));
                 wait(bar(kBarMmaDone), 0);
             }
         }
-    } else if (warp < 8) {
-        // ================================================= softmax
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
-        const int r = tid - 128;
+    } else {
+        // ================================================= softmax, two warpgroups
+        // Warpgroup ch (warps 4-7: ch = 0, warps 8-11: ch = 1) handles key tiles
+        // k = ch, ch + 2, ... with S buffer ch, O accumulator ch and its own
+        // running max m and sum l per row; warps 8-11 first rotate the queries.
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
+        const int ch = warp >= 8 ? 1 : 0;
+        const int r = (tid - 128) & 127;  // row = TMEM lane
         const int t = t0 + r / p.G;
         const int g = r % p.G;
-        const bool valid = t < t_end;
+        const bool valid = tile_valid && t < t_end;
+        if (ch == 1 && nt > 0) {
+            const int h = kvh * p.G + g;
+            // Rows past the last token (or of an absent tile) rotate a valid row and are never stored.
+            const int tt = valid ? t : pair_t0;
+            const int qp0 = query_pos(p.w, p.q_mode, tt);
+            rope_query_row<D>(Q + ((size_t)tt * p.H + h) * D, p.rope + (size_t)qp0 * (D / 2), p.q_scale,
+                              smem + L::kQ, smem + L::kQ + L::kQHalf, r);
+            fence_proxy_async_smem();  // generic stores -> read by the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lbar(kBarQReady));
+        }
         const int qp = valid ? query_pos(p.w, p.q_mode, t) : -1;
+        const uint32_t pfull_leader = lbar(kBarPFull0 + ch);
+        const uint32_t s_col = tmem + col_s(ch) + lane_off;
+        const uint32_t o_col = tmem + col_o(ch) + lane_off;
         float m_run = -INFINITY, l_run = 0.f;
         int npart = 0;
         bool ok = true;
-        for (int k = 0; k < nt; ++k) {
-            const int s = k & 1;
-            // Any failure so far (this wait, or an earlier O wait in any warp) ends
-            // the loop for all 128 threads together, so no thread is left waiting
-            // at a named barrier.
-            const bool w_ok = wait(bar(kBarSFull0 + s), (k >> 1) & 1);
-            if (!vote_all_ok_wg(w_ok && ok)) {
+        for (int k = ch; k < nt; k += 2) {
+            const int it = k >> 1;  // this warpgroup's iteration = phase of its S buffer
+            // Any failure so far ends the loop for all 128 threads of the warpgroup
+            // together, so none is left waiting at its named barrier.
+            const bool w_ok = wait(bar(kBarSFull0 + ch), it & 1);
+            if (!vote_all_ok(1 + ch, 128, w_ok && ok)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             uint32_t sr[4][32];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) tmem_ld32(tmem + col_s(s) + lane_off + 32 * h, sr[h]);
+            for (int h = 0; h < 4; ++h) tmem_ld32(s_col + 32 * h, sr[h]);
             tmem_wait_ld();
             const uint16_t ent = ctrl.list[kbeg + k];
             if (ent & 0x8000) {
                 // Elementwise streaming mask: key position of every column of the tile.
                 const int j = ent & 0x1FFF;
                 const int row = j * kTileRows + r;
-                int* kp = ctrl.kpos[npart & 1];
+                int* kp = ctrl.kpos[ch][npart & 1];
                 kp[r] = row < p.key_rows ? key_pos(p.w, row) : INT_MAX;
-                named_bar_sync(1, 128);
+                named_bar_sync(1 + ch, 128);
 #pragma unroll
                 for (int c4 = 0; c4 < 32; ++c4) {
                     const int4 k4 = *reinterpret_cast<const int4*>(kp + 4 * c4);
@@ -400,49 +467,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ++npart;
             }
-            float mt = -INFINITY;
+            // Row max with 8 independent partial maxima (no 128-long dependency chain).
+            float mx[8];
 #pragma unroll
-            for (int c = 0; c < 128; ++c) mt = fmaxf(mt, __uint_as_float(sr[c >> 5][c & 31]));
+            for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sr[0][i]);
+#pragma unroll
+            for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c >> 5][c & 31]));
+            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
             const float m_new = fmaxf(m_run, mt);
             const bool resc = m_new > m_run + kRescaleLog2;
             const float m_use = resc ? m_new : m_run;
             const float alpha = resc ? ex2_approx(m_run - m_use) : 1.f;
             const float base = (m_use == -INFINITY) ? 0.f : m_use;
-            float rs = 0.f;
+            const uint64_t base2 = f2pack(base, base);
+            uint64_t acc[4] = {0, 0, 0, 0};  // paired partial row sums
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int c2 = 0; c2 < 16; ++c2) {
-                    const float p0 = ex2_approx(__uint_as_float(sr[h][2 * c2]) - base);
-                    const float p1 = ex2_approx(__uint_as_float(sr[h][2 * c2 + 1]) - base);
-                    rs += p0 + p1;
+                    float d0, d1;
+                    f2unpack(sub2(f2pack(__uint_as_float(sr[h][2 * c2]), __uint_as_float(sr[h][2 * c2 + 1])), base2),
+                             d0, d1);
+                    const float p0 = ex2_approx(d0);
+                    const float p1 = ex2_approx(d1);
+                    acc[c2 & 3] = add2(acc[c2 & 3], f2pack(p0, p1));
                     pk[c2] = pack_f16x2(p0, p1);
                 }
-                asm volatile(
-                    "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-                    "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(tmem + col_s(s) + lane_off +
-                                                                                         16 * h),
-                    "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]), "r"(pk[7]),
-                    "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]), "r"(pk[13]), "r"(pk[14]),
-                    "r"(pk[15])
-                    : "memory");
+                tmem_st16(s_col + 16 * h, pk);  // P (fp16 pairs) over the first 64 columns of S
+            }
+            float rs;
+            {
+                const uint64_t a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+                float x0, x1;
+                f2unpack(add2(a01, a23), x0, x1);
+                rs = x0 + x1;
             }
             l_run = l_run * alpha + rs;
-            if (k > 0 && __any_sync(0xffffffffu, resc)) {
-                // O holds PV_0..PV_{k-1}; wait for the last of them, then rescale in TMEM.
-                bool o_ok = wait(bar(kBarOFull), (k - 1) & 1);
+            if (it > 0 && __any_sync(0xffffffffu, resc)) {
+                // O_ch holds this warpgroup's earlier PVs, the last of which (PV_{k-2})
+                // completed before QK_k was issued; rescale it in TMEM.
+                bool o_ok = wait(bar(kBarOFull0 + ch), (it - 1) & 1);
                 o_ok = __all_sync(0xffffffffu, o_ok);
                 if (o_ok) {
                     tc_fence_after();
 #pragma unroll 1
                     for (int cc = 0; cc < D / 32; ++cc) {
                         uint32_t o[32];
-                        tmem_ld32(tmem + kColO + lane_off + 32 * cc, o);
+                        tmem_ld32(o_col + 32 * cc, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tmem + kColO + lane_off + 32 * cc, o);
+                        tmem_st32(o_col + 32 * cc, o);
                     }
                 } else {
                     ok = false;
@@ -450,61 +527,68 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(kBarPFull0 + s));
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(pfull_leader);
             m_run = m_use;
         }
-        // ---- epilogue: O / l in fp32 (or the unnormalised split partials)
+        // ---- epilogue: merge the two warpgroups' (m, l, O) per row, then O / l in
+        // fp32 (or the unnormalised split partial), each warpgroup storing D/2 columns.
+        ctrl.red_m[ch][r] = m_run;
+        ctrl.red_l[ch][r] = l_run;
+        const bool all_ok = vote_all_ok(4, 256, ok);
+        const float m0 = ctrl.red_m[0][r], m1 = ctrl.red_m[1][r];
+        const float M = fmaxf(m0, m1);
+        // A side that saw no key for this row (or no tile at all) has m = -inf and
+        // an O that must not be read.
+        const bool use0 = m0 != -INFINITY, use1 = m1 != -INFINITY;
+        const float w0 = use0 ? ex2_approx(m0 - M) : 0.f;
+        const float w1 = use1 ? ex2_approx(m1 - M) : 0.f;
+        const float l_tot = w0 * ctrl.red_l[0][r] + w1 * ctrl.red_l[1][r];
         const size_t part_row = ((size_t)item_id * p.splits + split) * kTileRows + r;
-        if (ok && nt > 0) {
+        if (all_ok && nt > 0) {
             bool o_ok = wait(bar(kBarMmaDone), 0);  // single phase: after the last PV
             o_ok = __all_sync(0xffffffffu, o_ok);
             if (o_ok) {
                 tc_fence_after();
-                const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+                const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
                 const float sc = p.splits == 1 ? inv_l : 1.f;
-                float* dst = p.splits == 1 ? p.out + ((size_t)t * p.H + kvh * p.G + g) * D : p.part_o + part_row * D;
-                const bool store = p.splits > 1 || valid;
+                const float a0 = w0 * sc, a1 = w1 * sc;
+                float* dst = (p.splits == 1 ? p.out + ((size_t)t * p.H + kvh * p.G + g) * D : p.part_o + part_row * D) +
+                             ch * (D / 2);
+                const bool store = tile_valid && (p.splits > 1 || valid);
 #pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem + kColO + lane_off + 32 * cc, o);
+                for (int cc = 0; cc < D / 64; ++cc) {
+                    const uint32_t col = uint32_t(ch) * (D / 2) + 32 * cc;
+                    uint32_t o0[32], o1[32];
+                    tmem_ld32(tmem + kColO0 + lane_off + col, o0);
+                    tmem_ld32(tmem + kColO1 + lane_off + col, o1);
                     tmem_wait_ld();
                     if (store) {
+                        float v[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const float x0 = use0 ? __uint_as_float(o0[e]) * a0 : 0.f;
+                            const float x1 = use1 ? __uint_as_float(o1[e]) * a1 : 0.f;
+                            v[e] = x0 + x1;
+                        }
                         float4* d4 = reinterpret_cast<float4*>(dst + 32 * cc);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            d4[q] = make_float4(__uint_as_float(o[4 * q]) * sc, __uint_as_float(o[4 * q + 1]) * sc,
-                                                __uint_as_float(o[4 * q + 2]) * sc, __uint_as_float(o[4 * q + 3]) * sc);
+                        for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     }
                 }
-                if (p.splits > 1) p.part_ml[part_row] = make_float2(m_run, l_run);
+                if (p.splits > 1 && tile_valid && ch == 0) p.part_ml[part_row] = make_float2(M, l_tot);
             }
-        } else if (nt == 0 && p.splits > 1) {
+        } else if (nt == 0 && p.splits > 1 && tile_valid && ch == 0) {
             p.part_ml[part_row] = make_float2(-INFINITY, 0.f);
-        }
-    } else {
-        // ================================================= RoPE on Q (rows into TMEM)
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 192;");
-        const int r = tid - 256;
-        if (nt > 0) {
-            const int t = t0 + r / p.G;
-            const int h = kvh * p.G + r % p.G;
-            // Rows past the last token rotate a valid row (token t0) and are never stored.
-            const int tt = t < t_end ? t : t0;
-            const int qp = query_pos(p.w, p.q_mode, tt);
-            rope_query_row<D>(Q + ((size_t)tt * p.H + h) * D, p.rope + (size_t)qp * (D / 2), p.q_scale,
-                              tmem + kColQ + lane_off, tmem + kColQ + D / 2 + lane_off);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(kBarQReady));
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // neither CTA releases TMEM or exits while the pair's MMAs could touch it
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc_pair(tmem, kTmemCols);
     }
 }
 
@@ -571,7 +655,8 @@ cudaError_t launch_d(const AttnParams& p, const uint16_t* Q, const CUtensorMap& 
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    const unsigned grid = unsigned(p.Hkv * p.q_tiles * p.splits);
+    const int q_pairs = (p.q_tiles + 1) / 2;
+    const unsigned grid = unsigned(2 * q_pairs * p.Hkv * p.splits);
     stream_attn_kernel<D><<<grid, kThreads, smem, stream>>>(p, Q, tkh, tkl, tv16);
     return cudaGetLastError();
 }
