@@ -155,6 +155,32 @@ int fs_stream_attend_ext(fs_stream_t s, const void* Q_x, const void* K_x, const 
                          int n_x, void* out);
 
 /*
+ * fs_stream_attend_ext_static -- fs_stream_attend_ext without any allocation.
+ * The paper has no counterpart: this is a deployment variant for callers that
+ * may not allocate device memory per call (a drafting / verification loop
+ * under a device-memory budget fixed at start-up, where cudaMalloc / cudaFree
+ * could synchronise the device and stall a step).
+ *   Arguments, layouts, state rules and results are those of
+ *   fs_stream_attend_ext (out equal within rounding: the key range may be split
+ *   fewer times). The split-KV partials live in one fixed device array in the
+ *   library (64 partial tiles of 128 query rows: 4 MiB + 64 KiB), not in the
+ *   handle; no cudaMalloc, cudaFree or allocating library routine is called.
+ *   Limit: 2 * ceil(ceil(n_x * H/Hkv / 128) / 2) * Hkv <= 64 (at H/Hkv = 4 and
+ *   Hkv = 8: every n_x <= FS_MAX_VERIFY_TOKENS); larger calls fail with
+ *   FS_ERR_ARG and a message naming the limit, before any work is enqueued.
+ *   Set-up: the first call on a device looks up the array's address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture on the device.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents (nothing in it needs to start at zero: each call writes
+ *   every partial it reads). Calls that overlap on the GPU (other streams,
+ *   other handles) race on the array; serialise them.
+ * State: PREFILLED or STREAMING. Errors: FS_ERR_ARG, FS_ERR_STATE, FS_ERR_CUDA.
+ */
+int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x, const void* V_x,
+                                int n_x, void* out);
+
+/*
  * fs_stream_step_host -- one insert + attend with HOST buffers: copies K_new,
  * V_new and Q (bf16) to the device (staging buffers owned by the handle), runs
  * fs_stream_insert and fs_stream_attend, and copies out back, all enqueued on

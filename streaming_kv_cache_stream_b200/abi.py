@@ -44,6 +44,7 @@ SIGNATURES = {
     "fs_stream_insert": (_I, [_P, _P, _P]),
     "fs_stream_attend": (_I, [_P, _P, _P]),
     "fs_stream_attend_ext": (_I, [_P, _P, _P, _P, _I, _P]),
+    "fs_stream_attend_ext_static": (_I, [_P, _P, _P, _P, _I, _P]),
     "fs_stream_step_host": (_I, [_P, _P, _P, _P, _P]),
     "fs_stream_sync": (_I, [_P]),
     "fs_stream_info": (_I, [_P, ctypes.POINTER(fs_stream_info_t)]),
@@ -154,6 +155,12 @@ class Stream:
         self._bind_stream()
         _check(self._lib.fs_stream_attend_ext(self.handle, _ptr(Q_x), _ptr(K_x), _ptr(V_x), int(Q_x.shape[0]),
                                               _ptr(out, "float32")), self.handle)
+
+    def attend_ext_static(self, Q_x, K_x, V_x, out):
+        """attend_ext with the split-KV partials in the library's fixed device array (no allocation)."""
+        self._bind_stream()
+        _check(self._lib.fs_stream_attend_ext_static(self.handle, _ptr(Q_x), _ptr(K_x), _ptr(V_x),
+                                                     int(Q_x.shape[0]), _ptr(out, "float32")), self.handle)
 
     def step_host(self, K_new_h, V_new_h, Q_h, out_h):
         """Host-buffer step: numpy/torch CPU buffers (pinned for asynchrony)."""

@@ -113,5 +113,10 @@ cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_positions(const WindowShape& w, int rows, int* pos_out, cudaStream_t stream);
 cudaError_t launch_wait_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);
 size_t stream_attn_smem_bytes(int d);
+// Fixed split-KV scratch in device memory (no allocation): its capacity in
+// partial 128-row tiles, and its address on the current device (looked up on
+// the first call per device).
+int static_split_scratch_tiles();
+cudaError_t static_split_scratch(float** part_o, float2** part_ml);
 
 }  // namespace fs

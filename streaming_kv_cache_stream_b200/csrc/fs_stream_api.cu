@@ -398,6 +398,80 @@ int fs_stream_attend_ext(fs_stream_t s, const void* Q_x, const void* K_x, const 
     return do_attend(s, Q_x, out, n_x, fs::kQueryVerify, s->L + n_x);
 }
 
+// Same computation as fs_stream_attend_ext, with the split-KV partials in the
+// fixed device array of stream_attn.cu instead of the handle's scratch, and no
+// allocation on any path (the handle's buffers were allocated at create). The
+// split count is the one fs_stream_attend_ext would use, capped so the
+// partials fit the array; calls whose query tiles alone do not fit are
+// rejected. Callers: drafting / verification loops that run under a device
+// memory budget fixed at start-up and may not allocate per call (see
+// static_split_scratch in stream_attn.cu). The first call on a device looks
+// up the array's address (cudaGetSymbolAddress with that device current).
+int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x, const void* V_x, int n_x,
+                                void* out) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (!Q_x || !K_x || !V_x || !out) return fail(s, FS_ERR_ARG, "NULL tensor pointer");
+    if (!aligned16(Q_x) || !aligned16(K_x) || !aligned16(V_x) || !aligned16(out))
+        return fail(s, FS_ERR_ARG, "pointers must be 16-byte aligned");
+    if (n_x < 1 || n_x > FS_MAX_VERIFY_TOKENS) return fail(s, FS_ERR_ARG, "n_x must be in [1, %d]", FS_MAX_VERIFY_TOKENS);
+    if (Q_x == out) return fail(s, FS_ERR_ARG, "out must not alias Q_x");
+    if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "verify before the first insert");
+    const int key_rows = s->L + n_x;
+    const int q_tiles = (n_x * s->G + fs::kTileRows - 1) / fs::kTileRows;
+    // Partial tiles per split, counted as choose_splits does (query tiles padded to pairs).
+    const int tiles_padded = 2 * ((q_tiles + 1) / 2) * s->Hkv;
+    const int cap = fs::static_split_scratch_tiles();
+    if (tiles_padded > cap)
+        return fail(s, FS_ERR_ARG,
+                    "attend_ext_static: %d query tiles x %d kv heads need %d partial tiles per key split; "
+                    "the static split scratch holds %d",
+                    q_tiles, s->Hkv, tiles_padded, cap);
+    int splits = choose_splits(s, q_tiles, key_rows);
+    if (splits > cap / tiles_padded) splits = cap / tiles_padded;
+    float* part_o = nullptr;
+    float2* part_ml = nullptr;
+    FS_CUDA(s, fs::static_split_scratch(&part_o, &part_ml));
+    int rc = do_insert(s, K_x, V_x, n_x, 2);
+    if (rc) return rc;
+    AttnParams p;
+    p.w = shape_of(s);
+    p.key_rows = key_rows;
+    p.Hkv = s->Hkv;
+    p.G = s->G;
+    p.H = s->H;
+    p.d = s->d;
+    p.nq = n_x;
+    p.q_mode = fs::kQueryVerify;
+    p.q_tiles = q_tiles;
+    p.splits = splits;
+    p.q_scale = float(1.4426950408889634 / std::sqrt(double(s->d)));
+    p.rope = s->rope;
+    p.rope_rows = s->rope_rows;
+    p.out = static_cast<float*>(out);
+    p.part_o = part_o;
+    p.part_ml = part_ml;
+    p.err = s->err;
+    p.wait_limit_ns = s->wait_limit_ns;
+    fs::RopeParams rp;
+    rp.w = p.w;
+    rp.key_rows = key_rows;
+    rp.Hkv = s->Hkv;
+    rp.d = s->d;
+    rp.rope = s->rope;
+    rp.err = s->err;
+    rp.wait_limit_ns = s->wait_limit_ns;
+    FS_CUDA(s, fs::launch_kv_stream_rope(rp, s->tmap_k, s->tmap_v, s->tmap_kh, s->tmap_kl, s->tmap_v16, s->stream));
+    s->launches += 1;
+    FS_CUDA(s, fs::launch_stream_attn(p, static_cast<const uint16_t*>(Q_x), s->tmap_kh2, s->tmap_kl2, s->tmap_v16h,
+                                      s->stream));
+    s->launches += 1;
+    if (p.splits > 1) {
+        FS_CUDA(s, fs::launch_attn_combine(p, s->stream));
+        s->launches += 1;
+    }
+    return FS_OK;
+}
+
 int fs_stream_step_host(fs_stream_t s, const void* K_new_h, const void* V_new_h, const void* Q_h, void* out_h) {
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
     if (!K_new_h || !V_new_h || !Q_h || !out_h) return fail(s, FS_ERR_ARG, "NULL host pointer");

@@ -50,6 +50,7 @@
 // (head dims 64..127 in a second region), or 64-byte rows for V at D = 64.
 #include <cfloat>
 #include <climits>
+#include <mutex>
 
 #include "fs_internal.cuh"
 #include "sm100.cuh"
@@ -691,6 +692,54 @@ cudaError_t launch_positions(const WindowShape& w, int rows, int* pos_out, cudaS
 cudaError_t launch_wait_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream) {
     wait_probe_kernel<<<1, 32, 0, stream>>>(err, limit_ns);
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV scratch that needs no allocation (used by fs_stream_attend_ext_static).
+//
+// The split-KV path of stream_attn writes one partial (O, m, l) per query tile
+// and key split, then attn_combine merges them. fs_stream_attend_ext takes
+// that scratch from its handle (allocated at create and sized for the largest
+// call). This array serves callers that may not allocate device memory on a
+// per-call path: a drafting / verification loop with a device-memory budget
+// fixed at start-up, where a cudaMalloc or cudaFree (which can synchronise the
+// device and take unbounded time) would break the per-step latency budget.
+//
+// The array is file-scope device memory of fixed size (kStaticPartTiles
+// partial tiles of 128 rows: 64 x 128 x 128 x 4 B = 4 MiB of O plus 64 KiB of
+// (m, l) pairs). It is shared by every call on a device and keeps the last
+// call's contents; nothing in it has to start at zero, because every partial
+// row that attn_combine reads is written by the same call's stream_attn launch
+// first (including the (m = -inf, l = 0) rows of key splits with no visible
+// tile). Calls that overlap on the GPU (two streams, two handles) race on it.
+constexpr int kStaticPartTiles = 64;
+constexpr size_t kStaticPartOBytes = size_t(kStaticPartTiles) * kTileRows * 128 * sizeof(float);
+constexpr size_t kStaticPartMLBytes = size_t(kStaticPartTiles) * kTileRows * sizeof(float2);
+static __device__ __align__(256) unsigned char g_split_scratch[kStaticPartOBytes + kStaticPartMLBytes];
+
+int static_split_scratch_tiles() { return kStaticPartTiles; }
+
+cudaError_t static_split_scratch(float** part_o, float2** part_ml) {
+    // One symbol lookup per device, done by the first call on that device with
+    // the device current; later calls reuse the address.
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_split_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = ptr;
+    }
+    unsigned char* base = static_cast<unsigned char*>(addr[dev]);
+    *part_o = reinterpret_cast<float*>(base);
+    *part_ml = reinterpret_cast<float2*>(base + kStaticPartOBytes);
+    return cudaSuccess;
 }
 
 }  // namespace fs
