@@ -167,18 +167,19 @@ int do_insert(fs_stream_t s, const void* K, const void* V, int n_tokens, int mod
     return FS_OK;
 }
 
-// Splits of the key range per (kv head, pair of query tiles) so that small
-// query sets still fill the SMs (a pair occupies two); capped by the scratch
-// (one partial per query tile and split) and by the number of key tiles.
+// Splits of the key range per (kv head, unit of four query tiles) so that
+// small query sets still fill the SMs (a unit occupies a pair of SMs); capped
+// by the scratch (one partial per query tile and split) and by the number of
+// key tiles.
 int choose_splits(const fs_stream* s, int q_tiles, int key_rows) {
-    const int pairs = ((q_tiles + 1) / 2) * s->Hkv;
+    const int units = ((q_tiles + 3) / 4) * s->Hkv;
     const int slots = s->num_sms / 2;
-    if (pairs >= slots) return 1;
+    if (units >= slots) return 1;
     const int ktiles = (key_rows + fs::kTileRows - 1) / fs::kTileRows;
-    int sp = (slots + pairs - 1) / pairs;
+    int sp = (slots + units - 1) / units;
     if (sp > ktiles / 2) sp = ktiles / 2;
-    const int tiles_padded = 2 * pairs;
-    if (sp > s->part_rows_cap / tiles_padded) sp = s->part_rows_cap / tiles_padded;
+    const int tiles = q_tiles * s->Hkv;
+    if (sp > s->part_rows_cap / tiles) sp = s->part_rows_cap / tiles;
     return sp < 1 ? 1 : sp;
 }
 

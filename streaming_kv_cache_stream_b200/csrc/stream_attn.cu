@@ -8,33 +8,33 @@
 // q iff pos(q) <= pos(p)".
 //
 // Work unit: a pair of CTAs on two SMs (a cluster of 2, tcgen05 cta_group::2)
-// takes two 128-row query tiles of one kv head and runs M = 256 MMAs: each
-// CTA holds its own 128 query rows (Q in shared memory, S and O in its TMEM)
-// and half of every key tile (64 of the 128 keys) and V tile (D/2 of the
-// columns), so a key tile crosses the memory system once per pair. A query
-// tile packs 128/G tokens x the G query heads of one kv group (GQA). The keys
-// were rotated for this step by kv_stream_rope (at their shifted positions, as
-// fp16 hi + lo; V as fp16); this kernel rotates its query rows.
+// takes four 128-row query tiles of one kv head, as two query groups a and b
+// of M = 256 rows (each CTA holds 128 rows of each group). Every key tile is
+// staged once per pair (each CTA holds half of it: 64 of the 128 keys, D/2 of
+// the V columns) and multiplied against both groups, so the pair reads 96 KB
+// of operands per 512 query rows: on B200 the tensor pipes of all SMs would
+// otherwise need more from L2 than it delivers. A query tile packs 128/G
+// tokens x the G query heads of one kv group (GQA). The keys were rotated for
+// this step by kv_stream_rope (at their shifted positions, as fp16 hi + lo; V
+// as fp16); this kernel rotates its query rows.
 //
 // Warp roles per CTA (12 warps):
-//   warp 0      TMA producer: this CTA's halves of K hi/lo and V, 3 stages;
+//   warp 0      TMA producer: this CTA's halves of K hi/lo and V, 2 + 2 stages;
 //   warp 1      TMEM allocation; in the even CTA, the single MMA issuer;
-//   warps 4-7   softmax of the even key tiles (S buffer 0, O accumulator 0);
-//   warps 8-11  RoPE of the query rows into shared memory, then softmax of the
-//               odd key tiles (S buffer 1, O accumulator 1).
-// The two softmax warpgroups each keep their own running max and sum over
-// their half of the key tiles and their own O; the epilogue merges the two
-// (as a split of the key range would be merged). So they never wait for each
-// other, each has two MMA periods per tile, and the lazy O rescale never
-// stalls: QK of tile k already waits for PV of tile k-2, the last write to
-// the same O.
-// Pipeline: TMA K_j,V_j -> MMA S_j = Q K_j^T (into S_{j%2}) -> softmax ->
-// P_j (fp16, over S in TMEM) -> MMA O_{j%2} += P_j V_j; QK_{j+1} is issued
-// before PV_j.
+//   warps 4-7   group a: RoPE of its query rows, then its online softmax;
+//   warps 8-11  group b: the same.
+// TMEM per CTA: S_a, S_b (fp32 scores, 128 columns each; P as fp16 over the
+// first 64 columns of its S) and O_a, O_b (fp32, D columns each).
+// MMA issue order for key tile k: QK_a(k), PV_b(k-1), QK_b(k), PV_a(k). A QK
+// into S_g waits for the previous PV_g (it reads P_g from the same columns),
+// and that wait always has other work queued on the tensor pipe; while one
+// group's softmax runs, the tensor pipe works for the other group. A commit
+// of S_g(k) also orders the preceding PV_g(k-1), so the softmax may rescale
+// O_g in place before it hands over P_g(k).
 // Key tiles are walked in physical ring order; positions come from key_pos(),
 // so the ring never moves. Tiles whose every key is after the pair's last
-// query are skipped; tiles entirely visible to the pair skip the elementwise
-// mask.
+// query are skipped; per group, tiles entirely visible to it skip the
+// elementwise mask.
 //
 // Precision. Rotation happens in fp32 from the bf16 inputs and a table of
 // fp32 cos/sin evaluated in double. The rotated Q (pre-scaled by log2(e)/sqrt(d))
@@ -60,63 +60,63 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO0 = 256;         // O accumulators: 256 .. 256+D and 384 .. 384+D
-constexpr uint32_t kColO1 = 384;
 // Rescale O only when the running max grows by more than 2^14: P = 2^(s - m)
 // then stays below 2^14 (fp16 holds up to 65504), so most tiles skip it.
 constexpr float kRescaleLog2 = 14.0f;
-constexpr int kStages = 3;               // K and V operand stages per CTA
+constexpr int kKStages = 2;  // K hi/lo stages per CTA
+constexpr int kVStages = 2;  // V stages per CTA
 
-__device__ __forceinline__ constexpr uint32_t col_s(int s) { return s ? 128u : 0u; }
-__device__ __forceinline__ constexpr uint32_t col_o(int s) { return s ? kColO1 : kColO0; }
+__device__ __forceinline__ constexpr uint32_t col_s(int grp) { return grp ? 128u : 0u; }
+__device__ __forceinline__ constexpr uint32_t col_o(int grp) { return grp ? 384u : 256u; }
 
 enum : int {
-    kBarQReady = 0,
-    kBarKFull0 = 1,
-    kBarKEmpty0 = kBarKFull0 + kStages,
-    kBarVFull0 = kBarKEmpty0 + kStages,
-    kBarVEmpty0 = kBarVFull0 + kStages,
-    kBarSFull0 = kBarVEmpty0 + kStages,
-    kBarPFull0 = kBarSFull0 + 2,
-    kBarSFree0 = kBarPFull0 + 2,
-    kBarOFull0 = kBarSFree0 + 2,
-    kBarMmaDone = kBarOFull0 + 2,
+    kBarQReady0 = 0,                        // per group
+    kBarKFull0 = kBarQReady0 + 2,           // per K stage
+    kBarKEmpty0 = kBarKFull0 + kKStages,
+    kBarVFull0 = kBarKEmpty0 + kKStages,    // per V stage
+    kBarVEmpty0 = kBarVFull0 + kVStages,
+    kBarSFull0 = kBarVEmpty0 + kVStages,    // per group: QK done
+    kBarPFull0 = kBarSFull0 + 2,            // per group: P stored (and O rescaled)
+    kBarPVDone0 = kBarPFull0 + 2,           // per group: PV done (S free again)
+    kBarMmaDone = kBarPVDone0 + 2,
     kNumBars
 };
 
-constexpr uint8_t kSkip = 0, kFull = 1, kPartial = 2;
+constexpr int kMaskWords = kMaxKeyTiles / 32;
 
 struct Ctrl {
-    alignas(16) int kpos[2][2][kTileRows];  // [warpgroup][buffer][key]: positions of a masked tile's keys
-    float red_m[2][kTileRows];              // [warpgroup][row]: final running max (epilogue merge)
-    float red_l[2][kTileRows];              // [warpgroup][row]: final running sum
     uint64_t bars[kNumBars];
+    alignas(16) int kpos[2][kTileRows];  // per group: key positions of the tile being masked
+    uint32_t vis[kMaskWords];            // key tile visible to some query of the pair
+    uint32_t part[2][kMaskWords];        // per group: tile needs the elementwise mask
     uint32_t tmem_base;
-    int nvis;
-    uint16_t list[kMaxKeyTiles];  // visible tiles: bits 0-12 tile index, bit 15 partial
-    uint8_t cls[kMaxKeyTiles];
+    int j_begin;                         // first visible tile of this key split
+    int nt;                              // visible tiles in this key split
 };
+constexpr int kCtrlBytes = 2048;
+static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
 
-// Per-CTA shared memory: the CTA's 128 query rows as fp16 hi and lo (128-byte
-// swizzle, head dims 64..127 in a second region), then 3 stages, each with
-// this CTA's half of a key tile (64 of the 128 keys, K hi then K lo) and its
-// half of the V tile (all 128 keys, D/2 of the columns; 128-byte swizzle at
-// D = 128, 64-byte swizzle at D = 64).
+// Per-CTA shared memory after the control block (1024-byte aligned): the
+// CTA's 128 query rows of group a and of group b as fp16 hi and lo (128-byte
+// swizzle, head dims 64..127 in a second region), then the K stages (this
+// CTA's 64 keys of a tile, K hi then K lo), then the V stages (all 128 keys,
+// this CTA's D/2 columns; 128-byte swizzle at D = 128, 64-byte at D = 64).
+// At D = 128: 128 KB + 64 KB + 32 KB + 2 KB = 226 KB of the 227 KB per CTA.
 template <int D>
 struct Layout {
-    static constexpr int kQRegion = 128 * 128;               // 128 rows x 128 bytes
-    static constexpr int kQHalf = 128 * D * 2;               // one of Q hi / Q lo
-    static constexpr int kKRegion = 64 * 128;                // 64 key rows x 128 bytes
-    static constexpr int kKHalf = 64 * D * 2;                // one of K hi / K lo
+    static constexpr int kQRegion = 128 * 128;                // 128 rows x 128 bytes
+    static constexpr int kQHalf = 128 * D * 2;                // Q hi or Q lo of one group
+    static constexpr int kKRegion = 64 * 128;                 // 64 key rows x 128 bytes
+    static constexpr int kKHalf = 64 * D * 2;                 // K hi or K lo of a stage
     static constexpr int kKStage = 2 * kKHalf;
-    static constexpr int kVRow = D;                          // bytes per key row of the V half (D/2 x 2)
+    static constexpr int kVRow = D;                           // bytes per key row of the V half
     static constexpr int kVStage = kTileRows * kVRow;
-    static constexpr uint32_t kVLayout = D == 128 ? 2u : 4u; // 128- or 64-byte swizzle
-    static constexpr int kQ = 0;
-    static constexpr int kK0 = 2 * kQHalf;
-    static constexpr int kV0 = kK0 + kStages * kKStage;
-    static constexpr int kCtrl = kV0 + kStages * kVStage;
-    static constexpr int kBytes = kCtrl + int(sizeof(Ctrl));
+    static constexpr uint32_t kVLayout = D == 128 ? 2u : 4u;  // 128- or 64-byte swizzle
+    static constexpr int kQ = 0;                              // [group][hi, lo]
+    static constexpr int kK0 = 4 * kQHalf;
+    static constexpr int kV0 = kK0 + kKStages * kKStage;
+    static constexpr int kTiles = kV0 + kVStages * kVStage;
+    static constexpr int kSmemBytes = kCtrlBytes + kTiles;    // dynamic shared memory per CTA
 };
 
 // Lowest and highest window position among physical key rows [r0, r1). Rows of
@@ -218,58 +218,71 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+// Smallest visible key tile index >= j (the caller knows one exists).
+__device__ __forceinline__ int next_visible(const uint32_t* vis, int j) {
+    int w = j >> 5;
+    uint32_t bits = vis[w] & (0xFFFFFFFFu << (j & 31));
+    while (bits == 0 && w + 1 < kMaskWords) bits = vis[++w];
+    return bits ? (w << 5) + __ffs(bits) - 1 : j;
+}
+
+__device__ __forceinline__ bool test_bit(const uint32_t* m, int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
+
 template <int D>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     stream_attn_kernel(const __grid_constant__ AttnParams p, const uint16_t* __restrict__ Q,
                        const __grid_constant__ CUtensorMap tkh, const __grid_constant__ CUtensorMap tkl,
                        const __grid_constant__ CUtensorMap tv16) {
     using L = Layout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Ctrl& ctrl = *reinterpret_cast<Ctrl*>(smem + L::kCtrl);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    Ctrl& ctrl = *reinterpret_cast<Ctrl*>(smem_raw);
+    uint8_t* smem = smem_raw + kCtrlBytes;  // operand tiles
+    {
+        // Both CTAs of a pair see the same layout, so both leave here together.
+        uint32_t dyn;
+        asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+        if ((smem_u32(smem) & 1023u) != 0 || dyn < uint32_t(L::kSmemBytes)) {
+            if (threadIdx.x == 0) atomicOr(p.err, kErrBadLaunch);
+            return;
+        }
+    }
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const uint32_t rank = cluster_rank();  // 0: leader (issues the pair's MMAs), 1: peer
     const bool leader = rank == 0;
 
-    // ---- work item: a pair of query tiles (2 pq, 2 pq + 1) of one kv head; heavy
-    // pairs (later tokens see more keys) first.
+    // ---- work item: four query tiles 4u .. 4u+3 of one kv head (group a: 4u, 4u+1;
+    // group b: 4u+2, 4u+3; this CTA holds 4u + 2 grp + rank); heavy units first.
     const int pair_id = blockIdx.x >> 1;
     const int split = pair_id % p.splits;
     const int item = pair_id / p.splits;
-    const int q_pairs = (p.q_tiles + 1) >> 1;
-    const int pq = q_pairs - 1 - item / p.Hkv;
+    const int units = (p.q_tiles + 3) >> 2;
+    const int u = units - 1 - item / p.Hkv;
     const int kvh = item % p.Hkv;
-    const int qt = 2 * pq + int(rank);
-    const bool tile_valid = qt < p.q_tiles;
-    const int item_id = qt * p.Hkv + kvh;
-    const int tok_per_tile = kTileRows / p.G;
-    const int t0 = qt * tok_per_tile;
-    const int t_end = min(t0 + tok_per_tile, p.nq);
-    // Query-position range of the pair (the union of its valid tiles; positions grow with tokens).
-    const int pair_t0 = 2 * pq * tok_per_tile;
-    const int pair_t1 = min(pair_t0 + 2 * tok_per_tile, p.nq);
-    const int qmin = query_pos(p.w, p.q_mode, pair_t0);
-    const int qmax = query_pos(p.w, p.q_mode, pair_t1 - 1);
+    const int tpt = kTileRows / p.G;  // tokens per query tile
+    const int unit_t0 = 4 * u * tpt;
+    const int unit_t1 = min(unit_t0 + 4 * tpt, p.nq);
+    const int unit_qmax = query_pos(p.w, p.q_mode, unit_t1 - 1);
     const BoundedWait wait{p.err, p.wait_limit_ns, kErrTimeout};
 
     auto bar = [&](int i) { return smem_u32(&ctrl.bars[i]); };
     auto lbar = [&](int i) { return map_to_rank(smem_u32(&ctrl.bars[i]), 0); };  // the leader's copy
 
     if (tid == 0) {
-        mbar_init(bar(kBarQReady), 8);  // one arrival per RoPE warp of both CTAs
-        for (int s = 0; s < kStages; ++s) {
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(bar(kBarQReady0 + g), 8);  // one arrival per RoPE warp of the group, both CTAs
+            mbar_init(bar(kBarSFull0 + g), 1);
+            mbar_init(bar(kBarPFull0 + g), 8);   // one arrival per softmax warp of the group, both CTAs
+            mbar_init(bar(kBarPVDone0 + g), 1);
+        }
+        for (int s = 0; s < kKStages; ++s) {
             mbar_init(bar(kBarKFull0 + s), 1);
             mbar_init(bar(kBarKEmpty0 + s), 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
             mbar_init(bar(kBarVFull0 + s), 1);
             mbar_init(bar(kBarVEmpty0 + s), 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(kBarSFull0 + s), 1);
-            mbar_init(bar(kBarPFull0 + s), 8);  // one arrival per softmax warp of that buffer, both CTAs
-            mbar_init(bar(kBarSFree0 + s), 1);
-            mbar_init(bar(kBarOFull0 + s), 1);
         }
         mbar_init(bar(kBarMmaDone), 1);
         fence_mbar_init();
@@ -279,48 +292,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_relinquish_pair();
     }
 
-    // ---- classify key tiles against the pair's query range, then list the visible ones
+    // ---- classify key tiles against the unit's and each group's query range
     const int n_ktiles = (p.key_rows + kTileRows - 1) / kTileRows;
-    for (int j = tid; j < n_ktiles; j += kThreads) {
-        const int r0 = j * kTileRows;
-        const int r1 = min(r0 + kTileRows, p.key_rows);
-        int lo, hi;
-        key_bounds(p.w, r0, r1, lo, hi);
-        uint8_t c = kPartial;
-        if (lo > qmax) c = kSkip;
-        else if (hi <= qmin && r1 - r0 == kTileRows) c = kFull;
-        ctrl.cls[j] = c;
+    {
+        int gmin[2], gmax[2];
+        bool gpresent[2];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            const int t0 = unit_t0 + 2 * g * tpt;
+            const int t1 = min(t0 + 2 * tpt, p.nq);
+            gpresent[g] = t0 < t1;
+            gmin[g] = gpresent[g] ? query_pos(p.w, p.q_mode, t0) : 0;
+            gmax[g] = gpresent[g] ? query_pos(p.w, p.q_mode, t1 - 1) : 0;
+        }
+        const int words = (n_ktiles + 31) >> 5;
+        for (int wd = warp; wd < words; wd += kThreads / 32) {
+            const int j = wd * 32 + lane;
+            bool v = false, pa = true, pb = true;
+            if (j < n_ktiles) {
+                const int r0 = j * kTileRows;
+                const int r1 = min(r0 + kTileRows, p.key_rows);
+                int lo, hi;
+                key_bounds(p.w, r0, r1, lo, hi);
+                v = lo <= unit_qmax;
+                const bool full_tile = r1 - r0 == kTileRows;
+                pa = !(gpresent[0] && hi <= gmin[0] && full_tile);
+                pb = !(gpresent[1] && hi <= gmin[1] && full_tile);
+            }
+            const uint32_t bv = __ballot_sync(0xffffffffu, v);
+            const uint32_t ba = __ballot_sync(0xffffffffu, pa);
+            const uint32_t bb = __ballot_sync(0xffffffffu, pb);
+            if (lane == 0) {
+                ctrl.vis[wd] = bv;
+                ctrl.part[0][wd] = ba;
+                ctrl.part[1][wd] = bb;
+            }
+        }
+        (void)gmax;
     }
     __syncthreads();
-    if (warp == 0) {
-        int count = 0;
-        for (int base = 0; base < n_ktiles; base += 32) {
-            const int j = base + lane;
-            const uint8_t c = j < n_ktiles ? ctrl.cls[j] : kSkip;
-            const unsigned vis = __ballot_sync(0xffffffffu, c != kSkip);
-            if (c != kSkip) {
-                const int slot = count + __popc(vis & ((1u << lane) - 1u));
-                ctrl.list[slot] = uint16_t(j | (c == kPartial ? 0x8000 : 0));
+    if (tid == 0) {
+        // This split's share of the visible tiles: [kbeg, kend) in visible order.
+        const int words = (n_ktiles + 31) >> 5;
+        int nvis = 0;
+        for (int wd = 0; wd < words; ++wd) nvis += __popc(ctrl.vis[wd]);
+        const int kbeg = int((long long)split * nvis / p.splits);
+        const int kend = int((long long)(split + 1) * nvis / p.splits);
+        int j = 0, seen = 0;
+        for (int wd = 0; wd < words; ++wd) {
+            const int c = __popc(ctrl.vis[wd]);
+            if (seen + c > kbeg) {
+                uint32_t bits = ctrl.vis[wd];
+                for (int skip = kbeg - seen; skip > 0; --skip) bits &= bits - 1;
+                j = wd * 32 + __ffs(bits) - 1;
+                break;
             }
-            count += __popc(vis);
+            seen += c;
         }
-        if (lane == 0) ctrl.nvis = count;
+        ctrl.j_begin = j;
+        ctrl.nt = kend - kbeg;
     }
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or commit
     tc_fence_after();
     const uint32_t tmem = ctrl.tmem_base;
-    const int nvis = ctrl.nvis;
-    const int kbeg = int((long long)split * nvis / p.splits);
-    const int kend = int((long long)(split + 1) * nvis / p.splits);
-    const int nt = kend - kbeg;
+    const int nt = ctrl.nt;
+    const int j_begin = ctrl.j_begin;
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;  // TMEM lanes of this warp
 
     // Register split, one setmaxnreg per warpgroup at the head of its region:
-    // 128 x (80 + 208 + 208) <= 384 x 168, the registers allocated at launch.
+    // 128 x (96 + 200 + 200) <= 384 x 168, the registers allocated at launch.
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 96;");
         if (warp == 0) {
             // ============================================= TMA producer (both CTAs)
             // Each CTA loads its half of every operand tile: keys [64 r, 64 r + 64)
@@ -330,24 +374,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tma_prefetch_desc(&tkh);
                 tma_prefetch_desc(&tkl);
                 tma_prefetch_desc(&tv16);
+                int j = j_begin;
                 for (int k = 0; k < nt; ++k) {
-                    const int s = k % kStages;
-                    const uint32_t par = ((k / kStages) & 1) ^ 1;
-                    const int j = ctrl.list[kbeg + k] & 0x1FFF;
-                    if (!wait(bar(kBarKEmpty0 + s), par)) break;
-                    if (leader) mbar_arrive_expect_tx(bar(kBarKFull0 + s), 2 * L::kKStage);
-                    const uint32_t kd = smem_u32(smem + L::kK0 + s * L::kKStage);
+                    if (k > 0) j = next_visible(ctrl.vis, j + 1);
+                    const int ks = k % kKStages;
+                    if (!wait(bar(kBarKEmpty0 + ks), ((k / kKStages) & 1) ^ 1)) break;
+                    if (leader) mbar_arrive_expect_tx(bar(kBarKFull0 + ks), 2 * L::kKStage);
+                    const uint32_t kd = smem_u32(smem + L::kK0 + ks * L::kKStage);
 #pragma unroll
                     for (int r = 0; r < D / 64; ++r) {
                         tma_load_3d_pair(kd + r * L::kKRegion, &tkh, r * 64, j * kTileRows + 64 * int(rank), kvh,
-                                         lbar(kBarKFull0 + s));
+                                         lbar(kBarKFull0 + ks));
                         tma_load_3d_pair(kd + L::kKHalf + r * L::kKRegion, &tkl, r * 64,
-                                         j * kTileRows + 64 * int(rank), kvh, lbar(kBarKFull0 + s));
+                                         j * kTileRows + 64 * int(rank), kvh, lbar(kBarKFull0 + ks));
                     }
-                    if (!wait(bar(kBarVEmpty0 + s), par)) break;
-                    if (leader) mbar_arrive_expect_tx(bar(kBarVFull0 + s), 2 * L::kVStage);
-                    tma_load_3d_pair(smem_u32(smem + L::kV0 + s * L::kVStage), &tv16, (D / 2) * int(rank),
-                                     j * kTileRows, kvh, lbar(kBarVFull0 + s));
+                    const int vs = k % kVStages;
+                    if (!wait(bar(kBarVEmpty0 + vs), ((k / kVStages) & 1) ^ 1)) break;
+                    if (leader) mbar_arrive_expect_tx(bar(kBarVFull0 + vs), 2 * L::kVStage);
+                    tma_load_3d_pair(smem_u32(smem + L::kV0 + vs * L::kVStage), &tv16, (D / 2) * int(rank),
+                                     j * kTileRows, kvh, lbar(kBarVFull0 + vs));
                 }
             }
         } else if (warp == 1) {
@@ -357,89 +402,108 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 constexpr uint32_t idesc_pv = idesc_f16(256, D, false, false, false, true);
                 // Descriptors are formed once; a K step advances the start-address
                 // field (bits 0-13, in 16-byte units) by the step's offset.
-                const uint64_t dqh = sw128_desc(smem_u32(smem + L::kQ), 16, 1024);
-                const uint64_t dql = dqh + (L::kQHalf >> 4);
+                const uint64_t dq0 = sw128_desc(smem_u32(smem + L::kQ), 16, 1024);
                 const uint64_t dk0 = sw128_desc(smem_u32(smem + L::kK0), 16, 1024);
                 const uint64_t dv0 = smem_desc(smem_u32(smem + L::kV0), L::kVStage, 8 * L::kVRow, L::kVLayout);
-                bool ok = wait(bar(kBarQReady), 0);
-                for (int k = 0; ok && k <= nt; ++k) {
-                    if (k < nt) {
-                        const int s = k % kStages;
-                        const int sb = k & 1;
-                        if (!(ok = wait(bar(kBarKFull0 + s), (k / kStages) & 1))) break;
-                        if (k >= 2 && !(ok = wait(bar(kBarSFree0 + sb), ((k - 2) >> 1) & 1))) break;
-                        tc_fence_after();
-                        const uint64_t dkh = dk0 + uint32_t((s * L::kKStage) >> 4);
-                        const uint64_t dkl = dkh + (L::kKHalf >> 4);
-                        const uint32_t d_s = tmem + col_s(sb);
+                // S_g = Q_g K^T over the three hi/lo products.
+                auto issue_qk = [&](int grp, int ks) {
+                    const uint64_t dqh = dq0 + uint32_t((2 * grp * L::kQHalf) >> 4);
+                    const uint64_t dql = dqh + uint32_t(L::kQHalf >> 4);
+                    const uint64_t dkh = dk0 + uint32_t((ks * L::kKStage) >> 4);
+                    const uint64_t dkl = dkh + uint32_t(L::kKHalf >> 4);
+                    const uint32_t d_s = tmem + col_s(grp);
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t qo = ((kk >> 2) * L::kQRegion + (kk & 3) * 32) >> 4;
-                            const uint32_t ko = ((kk >> 2) * L::kKRegion + (kk & 3) * 32) >> 4;
-                            mma_ss_pair(d_s, dqh + qo, dkh + ko, idesc_qk, kk > 0);
-                            mma_ss_pair(d_s, dqh + qo, dkl + ko, idesc_qk, 1);
-                            mma_ss_pair(d_s, dql + qo, dkh + ko, idesc_qk, 1);
-                        }
-                        tc_commit_pair(bar(kBarSFull0 + sb));
-                        tc_commit_pair(bar(kBarKEmpty0 + s));
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t qo = ((kk >> 2) * L::kQRegion + (kk & 3) * 32) >> 4;
+                        const uint32_t ko = ((kk >> 2) * L::kKRegion + (kk & 3) * 32) >> 4;
+                        mma_ss_pair(d_s, dqh + qo, dkh + ko, idesc_qk, kk > 0);
+                        mma_ss_pair(d_s, dqh + qo, dkl + ko, idesc_qk, 1);
+                        mma_ss_pair(d_s, dql + qo, dkh + ko, idesc_qk, 1);
                     }
-                    if (k >= 1) {
-                        const int kp = k - 1;
-                        const int s = kp % kStages;
-                        const int sb = kp & 1;
-                        if (!(ok = wait(bar(kBarPFull0 + sb), (kp >> 1) & 1))) break;
-                        if (!(ok = wait(bar(kBarVFull0 + s), (kp / kStages) & 1))) break;
-                        tc_fence_after();
-                        const uint64_t dv = dv0 + uint32_t((s * L::kVStage) >> 4);
+                };
+                // O_g (+)= P_g V, P_g (fp16) from the first 64 columns of S_g.
+                auto issue_pv = [&](int grp, int vs, bool first) {
+                    const uint64_t dv = dv0 + uint32_t((vs * L::kVStage) >> 4);
 #pragma unroll
-                        for (int kk = 0; kk < kTileRows / 16; ++kk)
-                            mma_ts_pair(tmem + col_o(sb), tmem + col_s(sb) + kk * 8, dv + ((kk * 16 * L::kVRow) >> 4),
-                                        idesc_pv, (kp >= 2 || kk > 0));
-                        tc_commit_pair(bar(kBarVEmpty0 + s));
-                        tc_commit_pair(bar(kBarSFree0 + sb));
-                        tc_commit_pair(bar(kBarOFull0 + sb));
+                    for (int kk = 0; kk < kTileRows / 16; ++kk)
+                        mma_ts_pair(tmem + col_o(grp), tmem + col_s(grp) + kk * 8, dv + ((kk * 16 * L::kVRow) >> 4),
+                                    idesc_pv, (!first || kk > 0));
+                };
+                bool ok = wait(bar(kBarQReady0 + 0), 0) && wait(bar(kBarQReady0 + 1), 0);
+                for (int k = 0; ok && k <= nt; ++k) {
+                    const int ks = k % kKStages;
+                    if (k < nt) {
+                        if (!(ok = wait(bar(kBarKFull0 + ks), (k / kKStages) & 1))) break;
+                        if (k > 0 && !(ok = wait(bar(kBarPVDone0 + 0), (k - 1) & 1))) break;
+                        tc_fence_after();
+                        issue_qk(0, ks);
+                        tc_commit_pair(bar(kBarSFull0 + 0));
+                    }
+                    if (k > 0) {
+                        const int kp = k - 1;
+                        const int vs = kp % kVStages;
+                        if (!(ok = wait(bar(kBarPFull0 + 1), kp & 1))) break;
+                        tc_fence_after();
+                        issue_pv(1, vs, kp == 0);
+                        tc_commit_pair(bar(kBarPVDone0 + 1));
+                        tc_commit_pair(bar(kBarVEmpty0 + vs));
+                    }
+                    if (k < nt) {
+                        if (k > 0 && !(ok = wait(bar(kBarPVDone0 + 1), (k - 1) & 1))) break;
+                        tc_fence_after();
+                        issue_qk(1, ks);
+                        tc_commit_pair(bar(kBarSFull0 + 1));
+                        tc_commit_pair(bar(kBarKEmpty0 + ks));
+                        const int vs = k % kVStages;
+                        if (!(ok = wait(bar(kBarPFull0 + 0), k & 1))) break;
+                        if (!(ok = wait(bar(kBarVFull0 + vs), (k / kVStages) & 1))) break;
+                        tc_fence_after();
+                        issue_pv(0, vs, k == 0);
+                        tc_commit_pair(bar(kBarPVDone0 + 0));
                     }
                 }
-                // Drain: every MMA issued above completes before TMEM is released.
+                // Drain: every MMA issued above completes before TMEM is read or released.
                 tc_commit_pair(bar(kBarMmaDone));
                 wait(bar(kBarMmaDone), 0);
             }
         }
     } else {
-        // ================================================= softmax, two warpgroups
-        // Warpgroup ch (warps 4-7: ch = 0, warps 8-11: ch = 1) handles key tiles
-        // k = ch, ch + 2, ... with S buffer ch, O accumulator ch and its own
-        // running max m and sum l per row; warps 8-11 first rotate the queries.
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
-        const int ch = warp >= 8 ? 1 : 0;
+        // ================================================= query groups: RoPE, softmax, epilogue
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 200;");
+        const int grp = warp >= 8 ? 1 : 0;
         const int r = (tid - 128) & 127;  // row = TMEM lane
-        const int t = t0 + r / p.G;
-        const int g = r % p.G;
-        const bool valid = tile_valid && t < t_end;
-        if (ch == 1 && nt > 0) {
-            const int h = kvh * p.G + g;
+        const int qt = 4 * u + 2 * grp + int(rank);
+        const bool tile_valid = qt < p.q_tiles;
+        const int t = qt * tpt + r / p.G;
+        const int gh = r % p.G;           // query head within the kv group
+        const bool valid = tile_valid && t < p.nq;
+        if (nt > 0) {
             // Rows past the last token (or of an absent tile) rotate a valid row and are never stored.
-            const int tt = valid ? t : pair_t0;
+            const int tt = valid ? t : unit_t0;
             const int qp0 = query_pos(p.w, p.q_mode, tt);
-            rope_query_row<D>(Q + ((size_t)tt * p.H + h) * D, p.rope + (size_t)qp0 * (D / 2), p.q_scale,
-                              smem + L::kQ, smem + L::kQ + L::kQHalf, r);
+            uint8_t* qg = smem + L::kQ + 2 * grp * L::kQHalf;
+            rope_query_row<D>(Q + ((size_t)tt * p.H + kvh * p.G + gh) * D, p.rope + (size_t)qp0 * (D / 2), p.q_scale,
+                              qg, qg + L::kQHalf, r);
             fence_proxy_async_smem();  // generic stores -> read by the tensor core
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(lbar(kBarQReady));
+            if (lane == 0) mbar_arrive_cluster(lbar(kBarQReady0 + grp));
         }
         const int qp = valid ? query_pos(p.w, p.q_mode, t) : -1;
-        const uint32_t pfull_leader = lbar(kBarPFull0 + ch);
-        const uint32_t s_col = tmem + col_s(ch) + lane_off;
-        const uint32_t o_col = tmem + col_o(ch) + lane_off;
+        const uint32_t pfull_leader = lbar(kBarPFull0 + grp);
+        const uint32_t s_col = tmem + col_s(grp) + lane_off;
+        const uint32_t o_col = tmem + col_o(grp) + lane_off;
+        const uint32_t* part = ctrl.part[grp];
+        int* kp = ctrl.kpos[grp];
         float m_run = -INFINITY, l_run = 0.f;
-        int npart = 0;
         bool ok = true;
-        for (int k = ch; k < nt; k += 2) {
-            const int it = k >> 1;  // this warpgroup's iteration = phase of its S buffer
-            // Any failure so far ends the loop for all 128 threads of the warpgroup
-            // together, so none is left waiting at its named barrier.
-            const bool w_ok = wait(bar(kBarSFull0 + ch), it & 1);
-            if (!vote_all_ok(1 + ch, 128, w_ok && ok)) {
+        int j = j_begin;
+        for (int k = 0; k < nt; ++k) {
+            if (k > 0) j = next_visible(ctrl.vis, j + 1);
+            // Any failure so far ends the loop for all 128 threads of the group
+            // together, so none is left waiting at its named barrier. The vote is
+            // also the barrier that keeps kpos from being rewritten while read.
+            const bool w_ok = wait(bar(kBarSFull0 + grp), k & 1);
+            if (!vote_all_ok(1 + grp, 128, w_ok && ok)) {
                 ok = false;
                 break;
             }
@@ -448,14 +512,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int h = 0; h < 4; ++h) tmem_ld32(s_col + 32 * h, sr[h]);
             tmem_wait_ld();
-            const uint16_t ent = ctrl.list[kbeg + k];
-            if (ent & 0x8000) {
+            if (test_bit(part, j)) {
                 // Elementwise streaming mask: key position of every column of the tile.
-                const int j = ent & 0x1FFF;
                 const int row = j * kTileRows + r;
-                int* kp = ctrl.kpos[ch][npart & 1];
                 kp[r] = row < p.key_rows ? key_pos(p.w, row) : INT_MAX;
-                named_bar_sync(1 + ch, 128);
+                named_bar_sync(1 + grp, 128);
 #pragma unroll
                 for (int c4 = 0; c4 < 32; ++c4) {
                     const int4 k4 = *reinterpret_cast<const int4*>(kp + 4 * c4);
@@ -466,7 +527,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (k4.z > qp) q4[2] = ninf;
                     if (k4.w > qp) q4[3] = ninf;
                 }
-                ++npart;
             }
             // Row max with 8 independent partial maxima (no 128-long dependency chain).
             float mx[8];
@@ -506,24 +566,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 rs = x0 + x1;
             }
             l_run = l_run * alpha + rs;
-            if (it > 0 && __any_sync(0xffffffffu, resc)) {
-                // O_ch holds this warpgroup's earlier PVs, the last of which (PV_{k-2})
-                // completed before QK_k was issued; rescale it in TMEM.
-                bool o_ok = wait(bar(kBarOFull0 + ch), (it - 1) & 1);
-                o_ok = __all_sync(0xffffffffu, o_ok);
-                if (o_ok) {
-                    tc_fence_after();
+            if (k > 0 && __any_sync(0xffffffffu, resc)) {
+                // O_g holds the group's earlier PVs, the last of which completed
+                // before QK_g(k) was issued; rescale it in TMEM.
 #pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(o_col + 32 * cc, o);
-                        tmem_wait_ld();
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(o_col + 32 * cc, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(o_col + 32 * cc, o);
-                    }
-                } else {
-                    ok = false;
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(o_col + 32 * cc, o);
                 }
             }
             tmem_wait_st();
@@ -532,54 +585,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive_cluster(pfull_leader);
             m_run = m_use;
         }
-        // ---- epilogue: merge the two warpgroups' (m, l, O) per row, then O / l in
-        // fp32 (or the unnormalised split partial), each warpgroup storing D/2 columns.
-        ctrl.red_m[ch][r] = m_run;
-        ctrl.red_l[ch][r] = l_run;
-        const bool all_ok = vote_all_ok(4, 256, ok);
-        const float m0 = ctrl.red_m[0][r], m1 = ctrl.red_m[1][r];
-        const float M = fmaxf(m0, m1);
-        // A side that saw no key for this row (or no tile at all) has m = -inf and
-        // an O that must not be read.
-        const bool use0 = m0 != -INFINITY, use1 = m1 != -INFINITY;
-        const float w0 = use0 ? ex2_approx(m0 - M) : 0.f;
-        const float w1 = use1 ? ex2_approx(m1 - M) : 0.f;
-        const float l_tot = w0 * ctrl.red_l[0][r] + w1 * ctrl.red_l[1][r];
-        const size_t part_row = ((size_t)item_id * p.splits + split) * kTileRows + r;
-        if (all_ok && nt > 0) {
+        // ---- epilogue: O_g / l in fp32 (or the unnormalised split partial with (m, l))
+        const size_t part_row = (((size_t)qt * p.Hkv + kvh) * p.splits + split) * kTileRows + r;
+        if (ok && nt > 0) {
             bool o_ok = wait(bar(kBarMmaDone), 0);  // single phase: after the last PV
             o_ok = __all_sync(0xffffffffu, o_ok);
             if (o_ok) {
                 tc_fence_after();
-                const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
-                const float sc = p.splits == 1 ? inv_l : 1.f;
-                const float a0 = w0 * sc, a1 = w1 * sc;
-                float* dst = (p.splits == 1 ? p.out + ((size_t)t * p.H + kvh * p.G + g) * D : p.part_o + part_row * D) +
-                             ch * (D / 2);
+                const float sc = p.splits == 1 ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
+                float* dst = p.splits == 1 ? p.out + ((size_t)t * p.H + kvh * p.G + gh) * D : p.part_o + part_row * D;
                 const bool store = tile_valid && (p.splits > 1 || valid);
 #pragma unroll 1
-                for (int cc = 0; cc < D / 64; ++cc) {
-                    const uint32_t col = uint32_t(ch) * (D / 2) + 32 * cc;
-                    uint32_t o0[32], o1[32];
-                    tmem_ld32(tmem + kColO0 + lane_off + col, o0);
-                    tmem_ld32(tmem + kColO1 + lane_off + col, o1);
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(o_col + 32 * cc, o);
                     tmem_wait_ld();
                     if (store) {
-                        float v[32];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const float x0 = use0 ? __uint_as_float(o0[e]) * a0 : 0.f;
-                            const float x1 = use1 ? __uint_as_float(o1[e]) * a1 : 0.f;
-                            v[e] = x0 + x1;
-                        }
                         float4* d4 = reinterpret_cast<float4*>(dst + 32 * cc);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                        for (int q = 0; q < 8; ++q)
+                            d4[q] = make_float4(__uint_as_float(o[4 * q]) * sc, __uint_as_float(o[4 * q + 1]) * sc,
+                                                __uint_as_float(o[4 * q + 2]) * sc, __uint_as_float(o[4 * q + 3]) * sc);
                     }
                 }
-                if (p.splits > 1 && tile_valid && ch == 0) p.part_ml[part_row] = make_float2(M, l_tot);
+                if (p.splits > 1 && tile_valid) p.part_ml[part_row] = make_float2(m_run, l_run);
             }
-        } else if (nt == 0 && p.splits > 1 && tile_valid && ch == 0) {
+        } else if (nt == 0 && p.splits > 1 && tile_valid) {
             p.part_ml[part_row] = make_float2(-INFINITY, 0.f);
         }
     }
@@ -656,8 +687,8 @@ cudaError_t launch_d(const AttnParams& p, const uint16_t* Q, const CUtensorMap& 
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    const int q_pairs = (p.q_tiles + 1) / 2;
-    const unsigned grid = unsigned(2 * q_pairs * p.Hkv * p.splits);
+    const int units = (p.q_tiles + 3) / 4;
+    const unsigned grid = unsigned(2 * units * p.Hkv * p.splits);
     stream_attn_kernel<D><<<grid, kThreads, smem, stream>>>(p, Q, tkh, tkl, tv16);
     return cudaGetLastError();
 }
@@ -665,7 +696,7 @@ cudaError_t launch_d(const AttnParams& p, const uint16_t* Q, const CUtensorMap& 
 }  // namespace
 
 size_t stream_attn_smem_bytes(int d) {
-    const size_t need = size_t(d == 128 ? Layout<128>::kBytes : Layout<64>::kBytes) + 1024;
+    const size_t need = size_t(d == 128 ? Layout<128>::kSmemBytes : Layout<64>::kSmemBytes);
     // At least half the SM's shared memory, so two CTAs never compete for TMEM.
     return need < 120 * 1024 ? 120 * 1024 : need;
 }
