@@ -94,20 +94,23 @@ struct RopeParams {
     WindowShape w;
     int key_rows;         // rows per kv head to rotate
     int Hkv, d;
+    int rows_cap;         // rows allocated per kv head
     const float2* rope;   // [rope_rows][d/2] (cos, sin)
-    unsigned* err;
-    unsigned long long wait_limit_ns;
+    const uint16_t* K;    // bf16 cache [Hkv][rows_cap][d], pre-RoPE
+    const uint16_t* V;    // bf16 cache [Hkv][rows_cap][d]
+    uint16_t* Kh;         // fp16 rotated key, hi part, same layout
+    uint16_t* Kl;         // fp16 rotated key, lo part
+    uint16_t* V16;        // fp16 V
 };
 
 // Launchers (defined in the .cu files); all enqueue on `stream` and return the
 // launch's cudaError_t.
 cudaError_t launch_kv_stream_insert(const InsertParams& p, int num_sms, cudaStream_t stream);
-// kv_stream_rope: bf16 cache (tk, tv) -> fp16 rotated K hi (tkh), lo (tkl) and V (tv16).
-cudaError_t launch_kv_stream_rope(const RopeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
-                                  const CUtensorMap& tkh, const CUtensorMap& tkl, const CUtensorMap& tv16,
-                                  cudaStream_t stream);
-// stream_attn over the rotated operand cache (tkh, tkl, tv16).
-cudaError_t launch_stream_attn(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tkh,
+// kv_stream_rope: bf16 cache (K, V) -> fp16 rotated K hi, lo and fp16 V.
+cudaError_t launch_kv_stream_rope(const RopeParams& p, cudaStream_t stream);
+// stream_attn over the rotated operand cache (tkh, tkl, tv16); tq maps the
+// call's bf16 queries [nq][H][d] with box {64, G, 128/G} (128-byte swizzle).
+cudaError_t launch_stream_attn(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkh,
                                const CUtensorMap& tkl, const CUtensorMap& tv16, cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_positions(const WindowShape& w, int rows, int* pos_out, cudaStream_t stream);

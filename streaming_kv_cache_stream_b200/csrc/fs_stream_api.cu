@@ -46,8 +46,6 @@ struct fs_stream {
     int part_rows_cap = 0;  // rows of 128 query rows x d fp32 the split scratch holds
     void* stage = nullptr;  // host-path staging: K, V, Q, out
     size_t stage_bytes = 0;
-    CUtensorMap tmap_k, tmap_v;                 // bf16 cache, full 128-row tiles (rope loads)
-    CUtensorMap tmap_kh, tmap_kl, tmap_v16;     // fp16 operands, full tiles (rope stores)
     CUtensorMap tmap_kh2, tmap_kl2, tmap_v16h;  // fp16 operands, one CTA's half tile (attention loads)
     unsigned long long wait_limit_ns = 2000000000ull;
     long long cache_bytes = 0;
@@ -184,6 +182,11 @@ int choose_splits(const fs_stream* s, int q_tiles, int key_rows) {
 }
 
 int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key_rows) {
+    // Encoded before anything is enqueued, so a failure leaves no partial work.
+    CUtensorMap tq;  // this call's queries, one query tile (128/G tokens x G heads) per box
+    const int rcq = make_map(s, &tq, Q, s->d, s->H, nq, uint64_t(s->d) * 2, uint64_t(s->H) * s->d * 2, s->G,
+                             fs::kTileRows / s->G);
+    if (rcq) return rcq;
     const int q_tiles = (nq * s->G + fs::kTileRows - 1) / fs::kTileRows;
     AttnParams p;
     p.w = shape_of(s);
@@ -209,13 +212,16 @@ int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key
     rp.key_rows = key_rows;
     rp.Hkv = s->Hkv;
     rp.d = s->d;
+    rp.rows_cap = s->rows_cap;
     rp.rope = s->rope;
-    rp.err = s->err;
-    rp.wait_limit_ns = s->wait_limit_ns;
-    FS_CUDA(s, fs::launch_kv_stream_rope(rp, s->tmap_k, s->tmap_v, s->tmap_kh, s->tmap_kl, s->tmap_v16, s->stream));
+    rp.K = static_cast<const uint16_t*>(s->K_cache);
+    rp.V = static_cast<const uint16_t*>(s->V_cache);
+    rp.Kh = static_cast<uint16_t*>(s->Kh);
+    rp.Kl = static_cast<uint16_t*>(s->Kl);
+    rp.V16 = static_cast<uint16_t*>(s->V16);
+    FS_CUDA(s, fs::launch_kv_stream_rope(rp, s->stream));
     s->launches += 1;
-    FS_CUDA(s, fs::launch_stream_attn(p, static_cast<const uint16_t*>(Q), s->tmap_kh2, s->tmap_kl2, s->tmap_v16h,
-                                      s->stream));
+    FS_CUDA(s, fs::launch_stream_attn(p, tq, s->tmap_kh2, s->tmap_kl2, s->tmap_v16h, s->stream));
     s->launches += 1;
     if (p.splits > 1) {
         FS_CUDA(s, fs::launch_attn_combine(p, s->stream));
@@ -306,17 +312,8 @@ int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame,
         return bail(fail(nullptr, FS_ERR_CUDA, "RoPE table upload failed"));
 
     const uint64_t row_bytes = uint64_t(d) * 2;
-    int rc = make_map(nullptr, &s->tmap_k, s->K_cache, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
-                      fs::kTileRows, 1);
-    if (!rc) rc = make_map(nullptr, &s->tmap_v, s->V_cache, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
-                           fs::kTileRows, 1);
     const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (!rc) rc = make_map(nullptr, &s->tmap_kh, s->Kh, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
-                           fs::kTileRows, 1, f16);
-    if (!rc) rc = make_map(nullptr, &s->tmap_kl, s->Kl, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
-                           fs::kTileRows, 1, f16);
-    if (!rc) rc = make_map(nullptr, &s->tmap_v16, s->V16, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
-                           fs::kTileRows, 1, f16);
+    int rc = FS_OK;
     // Pair loads: 64 key rows of K hi / lo; all 128 key rows of d/2 V columns.
     if (!rc) rc = make_map(nullptr, &s->tmap_kh2, s->Kh, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
                            fs::kTileRows / 2, 1, f16);
@@ -432,6 +429,10 @@ int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x,
     float* part_o = nullptr;
     float2* part_ml = nullptr;
     FS_CUDA(s, fs::static_split_scratch(&part_o, &part_ml));
+    CUtensorMap tq;  // this call's queries, one query tile (128/G tokens x G heads) per box
+    const int rcq = make_map(s, &tq, Q_x, s->d, s->H, n_x, uint64_t(s->d) * 2, uint64_t(s->H) * s->d * 2, s->G,
+                             fs::kTileRows / s->G);
+    if (rcq) return rcq;
     int rc = do_insert(s, K_x, V_x, n_x, 2);
     if (rc) return rc;
     AttnParams p;
@@ -458,13 +459,16 @@ int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x,
     rp.key_rows = key_rows;
     rp.Hkv = s->Hkv;
     rp.d = s->d;
+    rp.rows_cap = s->rows_cap;
     rp.rope = s->rope;
-    rp.err = s->err;
-    rp.wait_limit_ns = s->wait_limit_ns;
-    FS_CUDA(s, fs::launch_kv_stream_rope(rp, s->tmap_k, s->tmap_v, s->tmap_kh, s->tmap_kl, s->tmap_v16, s->stream));
+    rp.K = static_cast<const uint16_t*>(s->K_cache);
+    rp.V = static_cast<const uint16_t*>(s->V_cache);
+    rp.Kh = static_cast<uint16_t*>(s->Kh);
+    rp.Kl = static_cast<uint16_t*>(s->Kl);
+    rp.V16 = static_cast<uint16_t*>(s->V16);
+    FS_CUDA(s, fs::launch_kv_stream_rope(rp, s->stream));
     s->launches += 1;
-    FS_CUDA(s, fs::launch_stream_attn(p, static_cast<const uint16_t*>(Q_x), s->tmap_kh2, s->tmap_kl2, s->tmap_v16h,
-                                      s->stream));
+    FS_CUDA(s, fs::launch_stream_attn(p, tq, s->tmap_kh2, s->tmap_kl2, s->tmap_v16h, s->stream));
     s->launches += 1;
     if (p.splits > 1) {
         FS_CUDA(s, fs::launch_attn_combine(p, s->stream));

@@ -79,6 +79,7 @@ enum : int {
     kBarPFull0 = kBarSFull0 + 2,            // per group: P stored (and O rescaled)
     kBarPVDone0 = kBarPFull0 + 2,           // per group: PV done (S free again)
     kBarMmaDone = kBarPVDone0 + 2,
+    kBarQLoad,                              // this CTA's bf16 query tiles landed (TMA)
     kNumBars
 };
 
@@ -152,46 +153,55 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 // the swizzled Q tiles `qhi` / `qlo` (the K-major A operand of the QK MMA).
 // Pair (i, i + D/2): for D = 128 chunk c of region 0 pairs with chunk c of
 // region 1; for D = 64 chunk c pairs with chunk c + 4.
-template <int D>
-__device__ __forceinline__ void rope_query_row(const uint16_t* __restrict__ qrow, const float2* __restrict__ cs,
-                                               float scale, uint8_t* qhi, uint8_t* qlo, int row) {
-    constexpr int kPairs = D / 16;
+template <int D, typename Ready>
+__device__ __forceinline__ void rope_query_row(const float2* __restrict__ cs, float scale, uint8_t* qhi, uint8_t* qlo,
+                                               int row, Ready ready) {
+    constexpr int kPairs = D / 16;  // 16-byte chunk pairs (c, c + D/16) of the row
+    constexpr int kHalf = kPairs / 2;
     const int sw = row & 7;
+    // The first half of the row's cos/sin is in flight while the query tile lands.
+    float4 t[kHalf][4];
 #pragma unroll
-    for (int c0 = 0; c0 < kPairs; c0 += 2) {
-        // Two chunk pairs per round: every load is issued before the arithmetic.
-        uint4 a[2], b[2];
-        float4 t[2][4];
+    for (int u = 0; u < kHalf; ++u)
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int c = c0 + u;
-            a[u] = __ldg(reinterpret_cast<const uint4*>(qrow + 8 * c));
-            b[u] = __ldg(reinterpret_cast<const uint4*>(qrow + D / 2 + 8 * c));
-            const float4* t4 = reinterpret_cast<const float4*>(cs + 8 * c);
+        for (int q = 0; q < 4; ++q) t[u][q] = __ldg(reinterpret_cast<const float4*>(cs + 8 * u) + q);
+    const bool ok = ready();  // on a timeout the rows rotate whatever is there; the error is reported
+    (void)ok;
+    // Read the whole bf16 row before overwriting its lo half in place.
+    uint4 a[kPairs], b[kPairs];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) t[u][q] = __ldg(t4 + q);
+    for (int c = 0; c < kPairs; ++c) {
+        const int oa = row * 128 + ((c ^ sw) << 4);
+        const int ob = D == 128 ? oa + Layout<D>::kQRegion : row * 128 + (((c + 4) ^ sw) << 4);
+        a[c] = *reinterpret_cast<const uint4*>(qlo + oa);
+        b[c] = *reinterpret_cast<const uint4*>(qlo + ob);
+    }
+#pragma unroll
+    for (int c = 0; c < kPairs; ++c) {
+        const int u = c % kHalf;
+        if (c == kHalf) {
+#pragma unroll
+            for (int v = 0; v < kHalf; ++v)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) t[v][q] = __ldg(reinterpret_cast<const float4*>(cs + 8 * (kHalf + v)) + q);
         }
+        const int oa = row * 128 + ((c ^ sw) << 4);
+        const int ob = D == 128 ? oa + Layout<D>::kQRegion : row * 128 + (((c + 4) ^ sw) << 4);
+        const uint32_t aw[4] = {a[c].x, a[c].y, a[c].z, a[c].w};
+        const uint32_t bw[4] = {b[c].x, b[c].y, b[c].z, b[c].w};
+        uint32_t ah[4], al[4], bh[4], bl[4];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int c = c0 + u;
-            const int oa = row * 128 + ((c ^ sw) << 4);
-            const int ob = D == 128 ? oa + Layout<D>::kQRegion : row * 128 + (((c + 4) ^ sw) << 4);
-            const uint32_t aw[4] = {a[u].x, a[u].y, a[u].z, a[u].w};
-            const uint32_t bw[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
-            uint32_t ah[4], al[4], bh[4], bl[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 tq = t[u][q];  // (cos, sin) of elements 8c + 2q and 8c + 2q + 1
-                const float x0 = bf16lo(aw[q]), x1 = bf16hi(aw[q]);
-                const float y0 = bf16lo(bw[q]), y1 = bf16hi(bw[q]);
-                split2((x0 * tq.x - y0 * tq.y) * scale, (x1 * tq.z - y1 * tq.w) * scale, ah[q], al[q]);
-                split2((y0 * tq.x + x0 * tq.y) * scale, (y1 * tq.z + x1 * tq.w) * scale, bh[q], bl[q]);
-            }
-            *reinterpret_cast<uint4*>(qhi + oa) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
-            *reinterpret_cast<uint4*>(qhi + ob) = make_uint4(bh[0], bh[1], bh[2], bh[3]);
-            *reinterpret_cast<uint4*>(qlo + oa) = make_uint4(al[0], al[1], al[2], al[3]);
-            *reinterpret_cast<uint4*>(qlo + ob) = make_uint4(bl[0], bl[1], bl[2], bl[3]);
+        for (int q = 0; q < 4; ++q) {
+            const float4 tq = t[u][q];  // (cos, sin) of elements 8c + 2q and 8c + 2q + 1
+            const float x0 = bf16lo(aw[q]), x1 = bf16hi(aw[q]);
+            const float y0 = bf16lo(bw[q]), y1 = bf16hi(bw[q]);
+            split2((x0 * tq.x - y0 * tq.y) * scale, (x1 * tq.z - y1 * tq.w) * scale, ah[q], al[q]);
+            split2((y0 * tq.x + x0 * tq.y) * scale, (y1 * tq.z + x1 * tq.w) * scale, bh[q], bl[q]);
         }
+        *reinterpret_cast<uint4*>(qhi + oa) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
+        *reinterpret_cast<uint4*>(qhi + ob) = make_uint4(bh[0], bh[1], bh[2], bh[3]);
+        *reinterpret_cast<uint4*>(qlo + oa) = make_uint4(al[0], al[1], al[2], al[3]);
+        *reinterpret_cast<uint4*>(qlo + ob) = make_uint4(bl[0], bl[1], bl[2], bl[3]);
     }
 }
 
@@ -230,7 +240,7 @@ __device__ __forceinline__ bool test_bit(const uint32_t* m, int j) { return (m[j
 
 template <int D>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    stream_attn_kernel(const __grid_constant__ AttnParams p, const uint16_t* __restrict__ Q,
+    stream_attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tq,
                        const __grid_constant__ CUtensorMap tkh, const __grid_constant__ CUtensorMap tkl,
                        const __grid_constant__ CUtensorMap tv16) {
     using L = Layout<D>;
@@ -285,86 +295,111 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(bar(kBarVEmpty0 + s), 1);
         }
         mbar_init(bar(kBarMmaDone), 1);
+        mbar_init(bar(kBarQLoad), 1);
         fence_mbar_init();
+        // This CTA's rows of both query groups, bf16, into the Q lo regions (the
+        // layout the rotation reads and overwrites in place); rows past the last
+        // token read as zero.
+        mbar_arrive_expect_tx(bar(kBarQLoad), 2 * L::kQHalf);
+#pragma unroll
+        for (int g = 0; g < 2; ++g)
+#pragma unroll
+            for (int reg = 0; reg < D / 64; ++reg)
+                tma_load_3d(smem_u32(smem + L::kQ + (2 * g + 1) * L::kQHalf + reg * L::kQRegion), &tq, 64 * reg,
+                            kvh * p.G, (4 * u + 2 * g + int(rank)) * tpt, bar(kBarQLoad));
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(&ctrl.tmem_base), kTmemCols);
         tmem_relinquish_pair();
     }
+    __syncthreads();  // barriers initialised before anyone waits on them
+    cluster_arrive();  // pairs with cluster_wait before the first cross-CTA operation
 
-    // ---- classify key tiles against the unit's and each group's query range
-    const int n_ktiles = (p.key_rows + kTileRows - 1) / kTileRows;
-    {
-        int gmin[2], gmax[2];
-        bool gpresent[2];
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            const int t0 = unit_t0 + 2 * g * tpt;
-            const int t1 = min(t0 + 2 * tpt, p.nq);
-            gpresent[g] = t0 < t1;
-            gmin[g] = gpresent[g] ? query_pos(p.w, p.q_mode, t0) : 0;
-            gmax[g] = gpresent[g] ? query_pos(p.w, p.q_mode, t1 - 1) : 0;
-        }
-        const int words = (n_ktiles + 31) >> 5;
-        for (int wd = warp; wd < words; wd += kThreads / 32) {
-            const int j = wd * 32 + lane;
-            bool v = false, pa = true, pb = true;
-            if (j < n_ktiles) {
-                const int r0 = j * kTileRows;
-                const int r1 = min(r0 + kTileRows, p.key_rows);
-                int lo, hi;
-                key_bounds(p.w, r0, r1, lo, hi);
-                v = lo <= unit_qmax;
-                const bool full_tile = r1 - r0 == kTileRows;
-                pa = !(gpresent[0] && hi <= gmin[0] && full_tile);
-                pb = !(gpresent[1] && hi <= gmin[1] && full_tile);
-            }
-            const uint32_t bv = __ballot_sync(0xffffffffu, v);
-            const uint32_t ba = __ballot_sync(0xffffffffu, pa);
-            const uint32_t bb = __ballot_sync(0xffffffffu, pb);
-            if (lane == 0) {
-                ctrl.vis[wd] = bv;
-                ctrl.part[0][wd] = ba;
-                ctrl.part[1][wd] = bb;
-            }
-        }
-        (void)gmax;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        // This split's share of the visible tiles: [kbeg, kend) in visible order.
-        const int words = (n_ktiles + 31) >> 5;
-        int nvis = 0;
-        for (int wd = 0; wd < words; ++wd) nvis += __popc(ctrl.vis[wd]);
-        const int kbeg = int((long long)split * nvis / p.splits);
-        const int kend = int((long long)(split + 1) * nvis / p.splits);
-        int j = 0, seen = 0;
-        for (int wd = 0; wd < words; ++wd) {
-            const int c = __popc(ctrl.vis[wd]);
-            if (seen + c > kbeg) {
-                uint32_t bits = ctrl.vis[wd];
-                for (int skip = kbeg - seen; skip > 0; --skip) bits &= bits - 1;
-                j = wd * 32 + __ffs(bits) - 1;
-                break;
-            }
-            seen += c;
-        }
-        ctrl.j_begin = j;
-        ctrl.nt = kend - kbeg;
-    }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or commit
-    tc_fence_after();
-    const uint32_t tmem = ctrl.tmem_base;
-    const int nt = ctrl.nt;
-    const int j_begin = ctrl.j_begin;
-    const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;  // TMEM lanes of this warp
-
+    // ---- prologue, split by warpgroup (each runs under its own register limit):
+    // warps 0-3 classify the key tiles against the unit's and each group's query
+    // range and place this split's share; warps 4-7 (group a) and 8-11 (group b)
+    // meanwhile rotate their query rows into shared memory.
     // Register split, one setmaxnreg per warpgroup at the head of its region:
     // 128 x (96 + 200 + 200) <= 384 x 168, the registers allocated at launch.
+    uint32_t tmem = 0;
+    int nt = 0, j_begin = 0;
+    const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;  // TMEM lanes of this warp
+    // The control block and the TMEM base are complete before anyone reads them
+    // (warps 0-3 publish them at named barrier 4 without waiting for the query
+    // rotation); both CTAs' barriers exist before any cross-CTA arrive or commit.
+    auto prologue_sync = [&](bool publisher) {
+        tc_fence_before();
+        if (publisher) asm volatile("bar.arrive 4, 384;" ::: "memory");
+        else named_bar_sync(4, 384);
+        cluster_wait();
+        tc_fence_after();
+        tmem = ctrl.tmem_base;
+        nt = ctrl.nt;
+        j_begin = ctrl.j_begin;
+    };
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 96;");
+        const int n_ktiles = (p.key_rows + kTileRows - 1) / kTileRows;
+        {
+            int gmin[2], gmax[2];
+            bool gpresent[2];
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                const int t0 = unit_t0 + 2 * g * tpt;
+                const int t1 = min(t0 + 2 * tpt, p.nq);
+                gpresent[g] = t0 < t1;
+                gmin[g] = gpresent[g] ? query_pos(p.w, p.q_mode, t0) : 0;
+                gmax[g] = gpresent[g] ? query_pos(p.w, p.q_mode, t1 - 1) : 0;
+            }
+            const int words = (n_ktiles + 31) >> 5;
+            for (int wd = warp; wd < words; wd += 4) {
+                const int j = wd * 32 + lane;
+                bool v = false, pa = true, pb = true;
+                if (j < n_ktiles) {
+                    const int r0 = j * kTileRows;
+                    const int r1 = min(r0 + kTileRows, p.key_rows);
+                    int lo, hi;
+                    key_bounds(p.w, r0, r1, lo, hi);
+                    v = lo <= unit_qmax;
+                    const bool full_tile = r1 - r0 == kTileRows;
+                    pa = !(gpresent[0] && hi <= gmin[0] && full_tile);
+                    pb = !(gpresent[1] && hi <= gmin[1] && full_tile);
+                }
+                const uint32_t bv = __ballot_sync(0xffffffffu, v);
+                const uint32_t ba = __ballot_sync(0xffffffffu, pa);
+                const uint32_t bb = __ballot_sync(0xffffffffu, pb);
+                if (lane == 0) {
+                    ctrl.vis[wd] = bv;
+                    ctrl.part[0][wd] = ba;
+                    ctrl.part[1][wd] = bb;
+                }
+            }
+            (void)gmax;
+        }
+        named_bar_sync(3, 128);  // warps 0-3: the masks are complete
+        if (tid == 0) {
+            // This split's share of the visible tiles: [kbeg, kend) in visible order.
+            const int words = (n_ktiles + 31) >> 5;
+            int nvis = 0;
+            for (int wd = 0; wd < words; ++wd) nvis += __popc(ctrl.vis[wd]);
+            const int kbeg = int((long long)split * nvis / p.splits);
+            const int kend = int((long long)(split + 1) * nvis / p.splits);
+            int j = 0, seen = 0;
+            for (int wd = 0; wd < words; ++wd) {
+                const int c = __popc(ctrl.vis[wd]);
+                if (seen + c > kbeg) {
+                    uint32_t bits = ctrl.vis[wd];
+                    for (int skip = kbeg - seen; skip > 0; --skip) bits &= bits - 1;
+                    j = wd * 32 + __ffs(bits) - 1;
+                    break;
+                }
+                seen += c;
+            }
+            ctrl.j_begin = j;
+            ctrl.nt = kend - kbeg;
+        }
+        named_bar_sync(3, 128);  // warps 0-3: the split is placed
+        prologue_sync(true);
         if (warp == 0) {
             // ============================================= TMA producer (both CTAs)
             // Each CTA loads its half of every operand tile: keys [64 r, 64 r + 64)
@@ -475,19 +510,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int qt = 4 * u + 2 * grp + int(rank);
         const bool tile_valid = qt < p.q_tiles;
         const int t = qt * tpt + r / p.G;
-        const int gh = r % p.G;           // query head within the kv group
-        const bool valid = tile_valid && t < p.nq;
-        if (nt > 0) {
-            // Rows past the last token (or of an absent tile) rotate a valid row and are never stored.
-            const int tt = valid ? t : unit_t0;
-            const int qp0 = query_pos(p.w, p.q_mode, tt);
+        {
+            // Rotate this group's query rows (landed by TMA) in shared memory while
+            // warps 0-3 classify the key tiles; rows past the last token rotate
+            // zeros and are never stored.
+            const int qp0 = query_pos(p.w, p.q_mode, (tile_valid && t < p.nq) ? t : unit_t0);
             uint8_t* qg = smem + L::kQ + 2 * grp * L::kQHalf;
-            rope_query_row<D>(Q + ((size_t)tt * p.H + kvh * p.G + gh) * D, p.rope + (size_t)qp0 * (D / 2), p.q_scale,
-                              qg, qg + L::kQHalf, r);
+            rope_query_row<D>(p.rope + (size_t)qp0 * (D / 2), p.q_scale, qg, qg + L::kQHalf, r,
+                              [&] { return wait(bar(kBarQLoad), 0); });
             fence_proxy_async_smem();  // generic stores -> read by the tensor core
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(lbar(kBarQReady0 + grp));
         }
+        prologue_sync(false);
+        const bool valid = tile_valid && t < p.nq;
+        if (nt > 0 && lane == 0) mbar_arrive_cluster(lbar(kBarQReady0 + grp));  // rows rotated in the prologue
         const int qp = valid ? query_pos(p.w, p.q_mode, t) : -1;
         const uint32_t pfull_leader = lbar(kBarPFull0 + grp);
         const uint32_t s_col = tmem + col_s(grp) + lane_off;
@@ -585,30 +620,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive_cluster(pfull_leader);
             m_run = m_use;
         }
-        // ---- epilogue: O_g / l in fp32 (or the unnormalised split partial with (m, l))
+        // ---- epilogue: O_g / l in fp32 (or the unnormalised split partial with (m, l)).
+        // The rows go through the group's Q region (free once every MMA is done),
+        // 16-byte chunk c of row r at chunk position c ^ (r & 7), and leave as
+        // whole contiguous rows per warp instruction.
         const size_t part_row = (((size_t)qt * p.Hkv + kvh) * p.splits + split) * kTileRows + r;
         if (ok && nt > 0) {
-            bool o_ok = wait(bar(kBarMmaDone), 0);  // single phase: after the last PV
-            o_ok = __all_sync(0xffffffffu, o_ok);
+            const bool o_ok = vote_all_ok(1 + grp, 128, wait(bar(kBarMmaDone), 0));  // single phase: after the last PV
             if (o_ok) {
                 tc_fence_after();
                 const float sc = p.splits == 1 ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
-                float* dst = p.splits == 1 ? p.out + ((size_t)t * p.H + kvh * p.G + gh) * D : p.part_o + part_row * D;
-                const bool store = tile_valid && (p.splits > 1 || valid);
+                uint8_t* stg = smem + L::kQ + 2 * grp * L::kQHalf;
+                constexpr int kRowBytes = D * 4;
 #pragma unroll 1
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t o[32];
                     tmem_ld32(o_col + 32 * cc, o);
                     tmem_wait_ld();
-                    if (store) {
-                        float4* d4 = reinterpret_cast<float4*>(dst + 32 * cc);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            d4[q] = make_float4(__uint_as_float(o[4 * q]) * sc, __uint_as_float(o[4 * q + 1]) * sc,
-                                                __uint_as_float(o[4 * q + 2]) * sc, __uint_as_float(o[4 * q + 3]) * sc);
+                    for (int q = 0; q < 8; ++q) {
+                        const int c = 8 * cc + q;
+                        *reinterpret_cast<float4*>(stg + r * kRowBytes + ((c ^ (r & 7)) << 4)) =
+                            make_float4(__uint_as_float(o[4 * q]) * sc, __uint_as_float(o[4 * q + 1]) * sc,
+                                        __uint_as_float(o[4 * q + 2]) * sc, __uint_as_float(o[4 * q + 3]) * sc);
                     }
                 }
                 if (p.splits > 1 && tile_valid) p.part_ml[part_row] = make_float2(m_run, l_run);
+                // Warp w of the group copies rows 32 w .. 32 w + 31; lane i works out the
+                // destination of row 32 w + i once and the copy loop broadcasts it.
+                const int row0 = (warp & 3) * 32;
+                float* dmy = nullptr;
+                {
+                    const int rr = row0 + lane;
+                    const int t2 = qt * tpt + rr / p.G;
+                    if (tile_valid && (p.splits > 1 || t2 < p.nq))
+                        dmy = p.splits == 1 ? p.out + ((size_t)t2 * p.H + kvh * p.G + rr % p.G) * D
+                                            : p.part_o + (part_row - r + rr) * D;
+                }
+                named_bar_sync(1 + grp, 128);
+                constexpr int kChunks = D / 4;              // 16-byte chunks per row
+                constexpr int kRowsPerInstr = 32 / kChunks;  // rows one warp instruction covers
+                const int c = lane % kChunks;
+#pragma unroll 8
+                for (int i = 0; i < 32; i += kRowsPerInstr) {
+                    const int il = i + lane / kChunks;
+                    float* drow = reinterpret_cast<float*>(
+                        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dmy), il));
+                    const int rr = row0 + il;
+                    const float4 v = *reinterpret_cast<const float4*>(stg + rr * kRowBytes + ((c ^ (rr & 7)) << 4));
+                    if (drow) reinterpret_cast<float4*>(drow)[c] = v;
+                }
             }
         } else if (nt == 0 && p.splits > 1 && tile_valid) {
             p.part_ml[part_row] = make_float2(-INFINITY, 0.f);
@@ -677,7 +738,7 @@ __global__ void wait_probe_kernel(unsigned* err, unsigned long long limit_ns) {
 }
 
 template <int D>
-cudaError_t launch_d(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tkh, const CUtensorMap& tkl,
+cudaError_t launch_d(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkh, const CUtensorMap& tkl,
                      const CUtensorMap& tv16, cudaStream_t stream) {
     const size_t smem = stream_attn_smem_bytes(D);
     static bool attr = false;
@@ -689,7 +750,7 @@ cudaError_t launch_d(const AttnParams& p, const uint16_t* Q, const CUtensorMap& 
     }
     const int units = (p.q_tiles + 3) / 4;
     const unsigned grid = unsigned(2 * units * p.Hkv * p.splits);
-    stream_attn_kernel<D><<<grid, kThreads, smem, stream>>>(p, Q, tkh, tkl, tv16);
+    stream_attn_kernel<D><<<grid, kThreads, smem, stream>>>(p, tq, tkh, tkl, tv16);
     return cudaGetLastError();
 }
 
@@ -701,9 +762,9 @@ size_t stream_attn_smem_bytes(int d) {
     return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
-cudaError_t launch_stream_attn(const AttnParams& p, const uint16_t* Q, const CUtensorMap& tkh,
+cudaError_t launch_stream_attn(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkh,
                                const CUtensorMap& tkl, const CUtensorMap& tv16, cudaStream_t stream) {
-    return p.d == 128 ? launch_d<128>(p, Q, tkh, tkl, tv16, stream) : launch_d<64>(p, Q, tkh, tkl, tv16, stream);
+    return p.d == 128 ? launch_d<128>(p, tq, tkh, tkl, tv16, stream) : launch_d<64>(p, tq, tkh, tkl, tv16, stream);
 }
 
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream) {
