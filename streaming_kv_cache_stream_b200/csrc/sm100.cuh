@@ -323,6 +323,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// Largest of three (sm_100 three-input form).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Paired fp32 arithmetic (sm_100): one instruction on two lanes of a 64-bit register.
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
     uint64_t r;

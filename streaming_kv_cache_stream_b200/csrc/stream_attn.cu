@@ -87,14 +87,15 @@ constexpr int kMaskWords = kMaxKeyTiles / 32;
 
 struct Ctrl {
     uint64_t bars[kNumBars];
-    alignas(16) int kpos[2][kTileRows];  // per group: key positions of the tile being masked
+    alignas(16) int kpos[kTileRows];     // key positions of the tile being masked
+    uint16_t red_m[2][2][kTileRows];     // [group][column half][row]: partial row max (bf16, rounded up)
     uint32_t vis[kMaskWords];            // key tile visible to some query of the pair
     uint32_t part[2][kMaskWords];        // per group: tile needs the elementwise mask
     uint32_t tmem_base;
     int j_begin;                         // first visible tile of this key split
     int nt;                              // visible tiles in this key split
 };
-constexpr int kCtrlBytes = 2048;
+constexpr int kCtrlBytes = 3072;
 static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
 
 // Per-CTA shared memory after the control block (1024-byte aligned): the
@@ -102,7 +103,7 @@ static_assert(sizeof(Ctrl) <= kCtrlBytes, "control block too large");
 // swizzle, head dims 64..127 in a second region), then the K stages (this
 // CTA's 64 keys of a tile, K hi then K lo), then the V stages (all 128 keys,
 // this CTA's D/2 columns; 128-byte swizzle at D = 128, 64-byte at D = 64).
-// At D = 128: 128 KB + 64 KB + 32 KB + 2 KB = 226 KB of the 227 KB per CTA.
+// At D = 128: 128 KB + 64 KB + 32 KB + 3 KB = 227 KB, all of a CTA's limit.
 template <int D>
 struct Layout {
     static constexpr int kQRegion = 128 * 128;                // 128 rows x 128 bytes
@@ -238,6 +239,14 @@ __device__ __forceinline__ int next_visible(const uint32_t* vis, int j) {
 
 __device__ __forceinline__ bool test_bit(const uint32_t* m, int j) { return (m[j >> 5] >> (j & 31)) & 1u; }
 
+// bf16 of x rounded toward +inf (-inf stays -inf), as raw bits.
+__device__ __forceinline__ uint16_t bf16_round_up(float x) {
+    uint32_t u = __float_as_uint(x);
+    if (x > 0.f) u += 0xFFFFu;
+    return uint16_t(u >> 16);
+}
+__device__ __forceinline__ float bf16_to_float(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
+
 template <int D>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     stream_attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tq,
@@ -283,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int g = 0; g < 2; ++g) {
             mbar_init(bar(kBarQReady0 + g), 8);  // one arrival per RoPE warp of the group, both CTAs
             mbar_init(bar(kBarSFull0 + g), 1);
-            mbar_init(bar(kBarPFull0 + g), 8);   // one arrival per softmax warp of the group, both CTAs
+            mbar_init(bar(kBarPFull0 + g), 16);  // one arrival per softmax warp (8 per CTA), both CTAs
             mbar_init(bar(kBarPVDone0 + g), 1);
         }
         for (int s = 0; s < kKStages; ++s) {
@@ -521,116 +530,147 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();  // generic stores -> read by the tensor core
         }
         prologue_sync(false);
-        const bool valid = tile_valid && t < p.nq;
         if (nt > 0 && lane == 0) mbar_arrive_cluster(lbar(kBarQReady0 + grp));  // rows rotated in the prologue
-        const int qp = valid ? query_pos(p.w, p.q_mode, t) : -1;
-        const uint32_t pfull_leader = lbar(kBarPFull0 + grp);
-        const uint32_t s_col = tmem + col_s(grp) + lane_off;
-        const uint32_t o_col = tmem + col_o(grp) + lane_off;
-        const uint32_t* part = ctrl.part[grp];
-        int* kp = ctrl.kpos[grp];
-        float m_run = -INFINITY, l_run = 0.f;
+
+        // ---- softmax: both warpgroups on every S tile of both groups; warpgroup
+        // hw takes columns [64 hw, 64 hw + 64) of the 128 keys (two warps per SM
+        // sub-partition on each tile). The halves agree on the row max through
+        // shared memory (each half's max rounded up to bf16, so both compute the
+        // same value; any base at or above the true max keeps P <= 1), keep their
+        // own partial row sums, and rescale their own D/2 columns of O.
+        const int hw = grp;                // column half (the warpgroup)
+        int qpos[2];                       // this row's query position in group g (-1: no query)
+        bool rvalid[2];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            const int qtg = 4 * u + 2 * g + int(rank);
+            const int tg = qtg * tpt + r / p.G;
+            rvalid[g] = qtg < p.q_tiles && tg < p.nq;
+            qpos[g] = rvalid[g] ? query_pos(p.w, p.q_mode, tg) : -1;
+        }
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
         bool ok = true;
         int j = j_begin;
-        for (int k = 0; k < nt; ++k) {
+        for (int k = 0; ok && k < nt; ++k) {
             if (k > 0) j = next_visible(ctrl.vis, j + 1);
-            // Any failure so far ends the loop for all 128 threads of the group
-            // together, so none is left waiting at its named barrier. The vote is
-            // also the barrier that keeps kpos from being rewritten while read.
-            const bool w_ok = wait(bar(kBarSFull0 + grp), k & 1);
-            if (!vote_all_ok(1 + grp, 128, w_ok && ok)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) tmem_ld32(s_col + 32 * h, sr[h]);
-            tmem_wait_ld();
-            if (test_bit(part, j)) {
-                // Elementwise streaming mask: key position of every column of the tile.
-                const int row = j * kTileRows + r;
-                kp[r] = row < p.key_rows ? key_pos(p.w, row) : INT_MAX;
-                named_bar_sync(1 + grp, 128);
-#pragma unroll
-                for (int c4 = 0; c4 < 32; ++c4) {
-                    const int4 k4 = *reinterpret_cast<const int4*>(kp + 4 * c4);
-                    const uint32_t ninf = __float_as_uint(-INFINITY);
-                    uint32_t* q4 = &sr[c4 >> 3][(c4 & 7) * 4];
-                    if (k4.x > qp) q4[0] = ninf;
-                    if (k4.y > qp) q4[1] = ninf;
-                    if (k4.z > qp) q4[2] = ninf;
-                    if (k4.w > qp) q4[3] = ninf;
+            const bool pa = test_bit(ctrl.part[0], j), pb = test_bit(ctrl.part[1], j);
+            if (pa || pb) {
+                // Key position of every column of the tile, for the elementwise
+                // streaming mask (the same key tile serves both groups).
+                if (hw == 0) {
+                    const int row = j * kTileRows + r;
+                    ctrl.kpos[r] = row < p.key_rows ? key_pos(p.w, row) : INT_MAX;
                 }
+                named_bar_sync(5, 256);
             }
-            // Row max with 8 independent partial maxima (no 128-long dependency chain).
-            float mx[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sr[0][i]);
+            for (int g = 0; g < 2; ++g) {
+                const uint32_t s_col = tmem + col_s(g) + lane_off + 64 * hw;
+                const bool w_ok = wait(bar(kBarSFull0 + g), k & 1);
+                tc_fence_after();
+                uint32_t sr[2][32];
+                tmem_ld32(s_col, sr[0]);
+                tmem_ld32(s_col + 32, sr[1]);
+                tmem_wait_ld();
+                if (g == 0 ? pa : pb) {
+                    const int qp = qpos[g];
 #pragma unroll
-            for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c >> 5][c & 31]));
-            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            const float m_new = fmaxf(m_run, mt);
-            const bool resc = m_new > m_run + kRescaleLog2;
-            const float m_use = resc ? m_new : m_run;
-            const float alpha = resc ? ex2_approx(m_run - m_use) : 1.f;
-            const float base = (m_use == -INFINITY) ? 0.f : m_use;
-            const uint64_t base2 = f2pack(base, base);
-            uint64_t acc[4] = {0, 0, 0, 0};  // paired partial row sums
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int c2 = 0; c2 < 16; ++c2) {
-                    float d0, d1;
-                    f2unpack(sub2(f2pack(__uint_as_float(sr[h][2 * c2]), __uint_as_float(sr[h][2 * c2 + 1])), base2),
-                             d0, d1);
-                    const float p0 = ex2_approx(d0);
-                    const float p1 = ex2_approx(d1);
-                    acc[c2 & 3] = add2(acc[c2 & 3], f2pack(p0, p1));
-                    pk[c2] = pack_f16x2(p0, p1);
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        const int4 k4 = *reinterpret_cast<const int4*>(ctrl.kpos + 64 * hw + 4 * c4);
+                        const uint32_t ninf = __float_as_uint(-INFINITY);
+                        uint32_t* q4 = &sr[c4 >> 3][(c4 & 7) * 4];
+                        if (k4.x > qp) q4[0] = ninf;
+                        if (k4.y > qp) q4[1] = ninf;
+                        if (k4.z > qp) q4[2] = ninf;
+                        if (k4.w > qp) q4[3] = ninf;
+                    }
                 }
-                tmem_st16(s_col + 16 * h, pk);  // P (fp16 pairs) over the first 64 columns of S
-            }
-            float rs;
-            {
-                const uint64_t a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
-                float x0, x1;
-                f2unpack(add2(a01, a23), x0, x1);
-                rs = x0 + x1;
-            }
-            l_run = l_run * alpha + rs;
-            if (k > 0 && __any_sync(0xffffffffu, resc)) {
-                // O_g holds the group's earlier PVs, the last of which completed
-                // before QK_g(k) was issued; rescale it in TMEM.
+                // Partial row max of this half: three-input max into 8 independent maxima.
+                float mx[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sr[0][i]);
+#pragma unroll
+                for (int c = 8; c < 64; c += 2)
+                    mx[(c >> 1) & 7] = fmax3(mx[(c >> 1) & 7], __uint_as_float(sr[c >> 5][c & 31]),
+                                             __uint_as_float(sr[c >> 5][(c + 1) & 31]));
+                const float mh = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+                ctrl.red_m[g][hw][r] = bf16_round_up(mh);
+                // Exchange point, and the uniform decision: a failed wait anywhere
+                // ends the loop for all 256 threads together.
+                if (!vote_all_ok(6, 256, w_ok && ok)) {
+                    ok = false;
+                    break;
+                }
+                const float mt = fmaxf(bf16_to_float(ctrl.red_m[g][0][r]), bf16_to_float(ctrl.red_m[g][1][r]));
+                const float m_new = fmaxf(m_run[g], mt);
+                const bool resc = m_new > m_run[g] + kRescaleLog2;
+                const float m_use = resc ? m_new : m_run[g];
+                const float alpha = resc ? ex2_approx(m_run[g] - m_use) : 1.f;
+                const float base = (m_use == -INFINITY) ? 0.f : m_use;
+                const uint64_t base2 = f2pack(base, base);
+                uint64_t acc[4] = {0, 0, 0, 0};  // paired partial row sums
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c2 = 0; c2 < 16; ++c2) {
+                        float d0, d1;
+                        f2unpack(sub2(f2pack(__uint_as_float(sr[h][2 * c2]), __uint_as_float(sr[h][2 * c2 + 1])),
+                                      base2),
+                                 d0, d1);
+                        const float p0 = ex2_approx(d0);
+                        const float p1 = ex2_approx(d1);
+                        acc[c2 & 3] = add2(acc[c2 & 3], f2pack(p0, p1));
+                        pk[c2] = pack_f16x2(p0, p1);
+                    }
+                    // P (fp16 pairs): keys 64 hw + 32 h .. + 31 -> packed columns 32 hw + 16 h ..
+                    tmem_st16(tmem + col_s(g) + lane_off + 32 * hw + 16 * h, pk);
+                }
+                float rs;
+                {
+                    const uint64_t a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+                    float x0, x1;
+                    f2unpack(add2(a01, a23), x0, x1);
+                    rs = x0 + x1;
+                }
+                l_run[g] = l_run[g] * alpha + rs;
+                if (k > 0 && __any_sync(0xffffffffu, resc)) {
+                    // O_g holds the group's earlier PVs, the last of which completed
+                    // before QK_g(k) was issued; rescale this half's columns in TMEM.
+                    const uint32_t o_col = tmem + col_o(g) + lane_off + uint32_t(hw) * (D / 2);
 #pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld32(o_col + 32 * cc, o);
-                    tmem_wait_ld();
+                    for (int cc = 0; cc < D / 64; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(o_col + 32 * cc, o);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(o_col + 32 * cc, o);
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(o_col + 32 * cc, o);
+                    }
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(lbar(kBarPFull0 + g));
+                m_run[g] = m_use;
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(pfull_leader);
-            m_run = m_use;
         }
-        // ---- epilogue: O_g / l in fp32 (or the unnormalised split partial with (m, l)).
-        // The rows go through the group's Q region (free once every MMA is done),
-        // 16-byte chunk c of row r at chunk position c ^ (r & 7), and leave as
-        // whole contiguous rows per warp instruction.
+        // ---- epilogue: warpgroup hw finishes group hw: O / l in fp32 (or the
+        // unnormalised split partial with (m, l)), l being the sum of the two
+        // halves' partial sums, exchanged through the (now free) K stages.
+        const int g = hw;  // qt, tile_valid above are this group's
         const size_t part_row = (((size_t)qt * p.Hkv + kvh) * p.splits + split) * kTileRows + r;
         if (ok && nt > 0) {
-            const bool o_ok = vote_all_ok(1 + grp, 128, wait(bar(kBarMmaDone), 0));  // single phase: after the last PV
-            if (o_ok) {
+            const bool mma_ok = wait(bar(kBarMmaDone), 0);  // single phase: after the last PV
+            float* red_l = reinterpret_cast<float*>(smem + L::kK0);  // [group][half][row]
+            red_l[(0 * 2 + hw) * kTileRows + r] = l_run[0];
+            red_l[(1 * 2 + hw) * kTileRows + r] = l_run[1];
+            if (vote_all_ok(6, 256, mma_ok)) {
                 tc_fence_after();
-                const float sc = p.splits == 1 ? (l_run > 0.f ? 1.f / l_run : 0.f) : 1.f;
-                uint8_t* stg = smem + L::kQ + 2 * grp * L::kQHalf;
+                const float l_tot = red_l[(g * 2 + 0) * kTileRows + r] + red_l[(g * 2 + 1) * kTileRows + r];
+                const float sc = p.splits == 1 ? (l_tot > 0.f ? 1.f / l_tot : 0.f) : 1.f;
+                const uint32_t o_col = tmem + col_o(g) + lane_off;
+                uint8_t* stg = smem + L::kQ + 2 * g * L::kQHalf;
                 constexpr int kRowBytes = D * 4;
 #pragma unroll 1
                 for (int cc = 0; cc < D / 32; ++cc) {
@@ -645,9 +685,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                         __uint_as_float(o[4 * q + 2]) * sc, __uint_as_float(o[4 * q + 3]) * sc);
                     }
                 }
-                if (p.splits > 1 && tile_valid) p.part_ml[part_row] = make_float2(m_run, l_run);
-                // Warp w of the group copies rows 32 w .. 32 w + 31; lane i works out the
-                // destination of row 32 w + i once and the copy loop broadcasts it.
+                if (p.splits > 1 && tile_valid) p.part_ml[part_row] = make_float2(m_run[g], l_tot);
+                // Warp w of the warpgroup copies rows 32 w .. 32 w + 31; lane i works
+                // out the destination of row 32 w + i once and the copy loop
+                // broadcasts it.
                 const int row0 = (warp & 3) * 32;
                 float* dmy = nullptr;
                 {
@@ -657,7 +698,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         dmy = p.splits == 1 ? p.out + ((size_t)t2 * p.H + kvh * p.G + rr % p.G) * D
                                             : p.part_o + (part_row - r + rr) * D;
                 }
-                named_bar_sync(1 + grp, 128);
+                named_bar_sync(1 + hw, 128);
                 constexpr int kChunks = D / 4;              // 16-byte chunks per row
                 constexpr int kRowsPerInstr = 32 / kChunks;  // rows one warp instruction covers
                 const int c = lane % kChunks;
@@ -674,6 +715,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         } else if (nt == 0 && p.splits > 1 && tile_valid) {
             p.part_ml[part_row] = make_float2(-INFINITY, 0.f);
         }
+        (void)rvalid;
     }
 
     tc_fence_before();
