@@ -4,8 +4,9 @@
 
 A step is one window step of the whole hot path over every layer of the
 workload: for each layer, kv_stream_insert of the new frame of each view plus
-the text (evicting each view's oldest frame), then stream_attn of the step's
-queries against the layer's cache. Default workload: the driving-shaped window
+the text (evicting each view's oldest frame; the same pass rotates every
+cached key at its new position), then stream_attn of the step's queries
+against the layer's cache. Default workload: the driving-shaped window
 (4 cameras x 4 frames x 180 tokens + 256 text tokens, 36 layers, H=32, Hkv=8,
 d=128), synthetic seeded inputs resident in HBM before timing.
 
@@ -321,7 +322,13 @@ def run_ours(args):
     value = world * fl_layer * layers / (ms_per_step * 1e-3) / 1e12
     att_avg_ms = statistics.mean(att_ms)
     att_tflops = fl_layer / (att_avg_ms * 1e-3) / 1e12
-    ins_bytes = 4.0 * wl.step_tokens * wl.Hkv * wl.d * 2  # read K_new, V_new + write both into the ring
+    # kv_stream_insert moves, per kv head: the step's new K/V rows (read from the
+    # caller, written into the ring), the other cached rows' K/V (read), and the
+    # rotated operands K hi, K lo, V fp16 of every row of the window's 128-row
+    # tiles (written). Cos/sin table reads (shared by all kv heads) are not counted.
+    L = wl.window_len
+    tiles_rows = (L + 127) // 128 * 128
+    ins_bytes = float(wl.Hkv * wl.d * 2 * (4 * wl.step_tokens + 2 * (L - wl.step_tokens) + 3 * tiles_rows))
     ins_avg_ms = statistics.mean(ins_ms)
     peaks, src = load_peaks()
     peak_t = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))

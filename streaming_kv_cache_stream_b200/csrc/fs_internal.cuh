@@ -78,36 +78,28 @@ struct AttnParams {
 };
 
 struct InsertParams {
-    const uint4* K_src;   // [N][Hkv][d] bf16 as 16-byte chunks
-    const uint4* V_src;
-    uint4* K_cache;       // [Hkv][rows_cap][d]
-    uint4* V_cache;
-    int N;                // tokens to insert
-    int Hkv;
-    int chunks;           // d * 2 / 16 chunks per (token, kv head) vector
-    int rows_cap;         // rows per kv head in the cache
-    int mode;             // 0: prefill (row = t), 1: step, 2: drafted block (row = L + t)
-    int V, T, n, X, ring_rows, head;
-};
-
-struct RopeParams {
-    WindowShape w;
-    int key_rows;         // rows per kv head to rotate
-    int Hkv, d;
-    int rows_cap;         // rows allocated per kv head
-    const float2* rope;   // [rope_rows][d/2] (cos, sin)
-    const uint16_t* K;    // bf16 cache [Hkv][rows_cap][d], pre-RoPE
-    const uint16_t* V;    // bf16 cache [Hkv][rows_cap][d]
-    uint16_t* Kh;         // fp16 rotated key, hi part, same layout
-    uint16_t* Kl;         // fp16 rotated key, lo part
-    uint16_t* V16;        // fp16 V
+    WindowShape w;          // the window after this insert (head advanced): key positions
+    int mode;               // 0: prefill (row = t), 1: step, 2: drafted block (row = L + t)
+    int old_head;           // step: the ring slot each view's new frame overwrites
+    int N;                  // tokens in K_src / V_src
+    int row_begin, row_end; // physical rows processed (whole 128-row tiles, within rows_cap)
+    int key_rows;           // rows [0, key_rows) hold keys; later rows get zero operands
+    int Hkv, d, rows_cap;
+    const uint16_t* K_src;  // [N][Hkv][d] bf16, pre-RoPE
+    const uint16_t* V_src;
+    uint16_t* K;            // bf16 cache [Hkv][rows_cap][d]: new rows written, others read
+    uint16_t* V;
+    const float2* rope;     // [rope_rows][d/2] (cos, sin)
+    uint16_t* Kh;           // fp16 rotated key, hi part, same layout as the cache
+    uint16_t* Kl;           // fp16 rotated key, lo part
+    uint16_t* V16;          // fp16 V
 };
 
 // Launchers (defined in the .cu files); all enqueue on `stream` and return the
 // launch's cudaError_t.
-cudaError_t launch_kv_stream_insert(const InsertParams& p, int num_sms, cudaStream_t stream);
-// kv_stream_rope: bf16 cache (K, V) -> fp16 rotated K hi, lo and fp16 V.
-cudaError_t launch_kv_stream_rope(const RopeParams& p, cudaStream_t stream);
+// kv_stream_insert: new K/V into the bf16 cache, and every processed row's rotated
+// fp16 K hi / lo and fp16 V.
+cudaError_t launch_kv_stream_insert(const InsertParams& p, cudaStream_t stream);
 // stream_attn over the rotated operand cache (tkh, tkl, tv16); tq maps the
 // call's bf16 queries [nq][H][d] with box {64, G, 128/G} (128-byte swizzle).
 cudaError_t launch_stream_attn(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkh,

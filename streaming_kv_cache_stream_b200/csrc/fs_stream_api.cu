@@ -143,24 +143,34 @@ int check_err_word(fs_stream_t s) {
     return FS_OK;
 }
 
-int do_insert(fs_stream_t s, const void* K, const void* V, int n_tokens, int mode) {
+// One fused pass (kernel kv_stream_insert): this call's K/V into the cache and
+// every row of the processed range rotated at its position in the window as it
+// stands after the insert (new_head). Prefill and step process every key tile;
+// a drafted block only the tiles from L on (the window's rows were rotated by
+// the last insert and have not moved since).
+int do_insert(fs_stream_t s, const void* K, const void* V, int n_tokens, int mode, int new_head) {
     InsertParams p;
-    p.K_src = static_cast<const uint4*>(K);
-    p.V_src = static_cast<const uint4*>(V);
-    p.K_cache = reinterpret_cast<uint4*>(s->K_cache);
-    p.V_cache = reinterpret_cast<uint4*>(s->V_cache);
-    p.N = n_tokens;
-    p.Hkv = s->Hkv;
-    p.chunks = s->d * 2 / 16;
-    p.rows_cap = s->rows_cap;
+    p.w = shape_of(s);
+    p.w.head = new_head;
     p.mode = mode;
-    p.V = s->V;
-    p.T = s->T;
-    p.n = s->n;
-    p.X = s->X;
-    p.ring_rows = s->ring_rows;
-    p.head = s->head;
-    FS_CUDA(s, fs::launch_kv_stream_insert(p, s->num_sms, s->stream));
+    p.old_head = s->head;
+    p.N = n_tokens;
+    p.key_rows = mode == 2 ? s->L + n_tokens : s->L;
+    p.row_begin = mode == 2 ? s->L / fs::kTileRows * fs::kTileRows : 0;
+    p.row_end = (p.key_rows + fs::kTileRows - 1) / fs::kTileRows * fs::kTileRows;
+    if (p.row_end > s->rows_cap) p.row_end = s->rows_cap;
+    p.Hkv = s->Hkv;
+    p.d = s->d;
+    p.rows_cap = s->rows_cap;
+    p.K_src = static_cast<const uint16_t*>(K);
+    p.V_src = static_cast<const uint16_t*>(V);
+    p.K = s->K_cache;
+    p.V = s->V_cache;
+    p.rope = s->rope;
+    p.Kh = s->Kh;
+    p.Kl = s->Kl;
+    p.V16 = s->V16;
+    FS_CUDA(s, fs::launch_kv_stream_insert(p, s->stream));
     s->launches += 1;
     return FS_OK;
 }
@@ -207,20 +217,6 @@ int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key
     p.part_ml = s->part_ml;
     p.err = s->err;
     p.wait_limit_ns = s->wait_limit_ns;
-    fs::RopeParams rp;
-    rp.w = p.w;
-    rp.key_rows = key_rows;
-    rp.Hkv = s->Hkv;
-    rp.d = s->d;
-    rp.rows_cap = s->rows_cap;
-    rp.rope = s->rope;
-    rp.K = static_cast<const uint16_t*>(s->K_cache);
-    rp.V = static_cast<const uint16_t*>(s->V_cache);
-    rp.Kh = static_cast<uint16_t*>(s->Kh);
-    rp.Kl = static_cast<uint16_t*>(s->Kl);
-    rp.V16 = static_cast<uint16_t*>(s->V16);
-    FS_CUDA(s, fs::launch_kv_stream_rope(rp, s->stream));
-    s->launches += 1;
     FS_CUDA(s, fs::launch_stream_attn(p, tq, s->tmap_kh2, s->tmap_kl2, s->tmap_v16h, s->stream));
     s->launches += 1;
     if (p.splits > 1) {
@@ -356,14 +352,14 @@ int fs_stream_insert(fs_stream_t s, const void* K_new, const void* V_new) {
     if (!aligned16(K_new) || !aligned16(V_new)) return fail(s, FS_ERR_ARG, "K_new/V_new must be 16-byte aligned");
     if (s->state == FS_STATE_EXPECT_PREFILL) {
         s->head = 0;
-        int rc = do_insert(s, K_new, V_new, s->L, 0);
+        int rc = do_insert(s, K_new, V_new, s->L, 0, 0);
         if (rc) return rc;
         for (int f = 0; f < s->T; ++f) s->slot_frame[f] = f;
         s->state = FS_STATE_PREFILLED;
         s->last_insert_tokens = s->L;
         return FS_OK;
     }
-    int rc = do_insert(s, K_new, V_new, s->step_tokens, 1);
+    int rc = do_insert(s, K_new, V_new, s->step_tokens, 1, (s->head + 1) % s->T);
     if (rc) return rc;
     s->slot_frame[s->head] = (long long)s->T + s->steps;  // the k-th step inserts frame T-1+k
     s->head = (s->head + 1) % s->T;
@@ -391,7 +387,7 @@ int fs_stream_attend_ext(fs_stream_t s, const void* Q_x, const void* K_x, const 
     if (n_x < 1 || n_x > FS_MAX_VERIFY_TOKENS) return fail(s, FS_ERR_ARG, "n_x must be in [1, %d]", FS_MAX_VERIFY_TOKENS);
     if (Q_x == out) return fail(s, FS_ERR_ARG, "out must not alias Q_x");
     if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "verify before the first insert");
-    int rc = do_insert(s, K_x, V_x, n_x, 2);
+    int rc = do_insert(s, K_x, V_x, n_x, 2, s->head);
     if (rc) return rc;
     return do_attend(s, Q_x, out, n_x, fs::kQueryVerify, s->L + n_x);
 }
@@ -433,7 +429,7 @@ int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x,
     const int rcq = make_map(s, &tq, Q_x, s->d, s->H, n_x, uint64_t(s->d) * 2, uint64_t(s->H) * s->d * 2, s->G,
                              fs::kTileRows / s->G);
     if (rcq) return rcq;
-    int rc = do_insert(s, K_x, V_x, n_x, 2);
+    int rc = do_insert(s, K_x, V_x, n_x, 2, s->head);
     if (rc) return rc;
     AttnParams p;
     p.w = shape_of(s);
@@ -454,20 +450,6 @@ int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x,
     p.part_ml = part_ml;
     p.err = s->err;
     p.wait_limit_ns = s->wait_limit_ns;
-    fs::RopeParams rp;
-    rp.w = p.w;
-    rp.key_rows = key_rows;
-    rp.Hkv = s->Hkv;
-    rp.d = s->d;
-    rp.rows_cap = s->rows_cap;
-    rp.rope = s->rope;
-    rp.K = static_cast<const uint16_t*>(s->K_cache);
-    rp.V = static_cast<const uint16_t*>(s->V_cache);
-    rp.Kh = static_cast<uint16_t*>(s->Kh);
-    rp.Kl = static_cast<uint16_t*>(s->Kl);
-    rp.V16 = static_cast<uint16_t*>(s->V16);
-    FS_CUDA(s, fs::launch_kv_stream_rope(rp, s->stream));
-    s->launches += 1;
     FS_CUDA(s, fs::launch_stream_attn(p, tq, s->tmap_kh2, s->tmap_kl2, s->tmap_v16h, s->stream));
     s->launches += 1;
     if (p.splits > 1) {
