@@ -428,6 +428,113 @@ def run_ours(args):
     return result
 
 
+def run_verify(args):
+    """Drafted-block verify calls (workload 5): fs_stream_attend_ext of 8-token
+    blocks against the medium window's cache after one step, inputs resident;
+    a "step" is one verify call. The e2e leg copies each block from pinned host
+    memory and the output back inside the timed region."""
+    import numpy as np
+    import torch
+
+    from streaming_kv_cache_stream_b200.abi import Stream, load
+    from streaming_kv_cache_stream_b200.inputs import WORKLOADS, verify_inputs, window_inputs
+
+    world, rank, local = dist_setup(args.gpus)
+    load()
+    wid = args.workload
+    wl = WORKLOADS[wid]
+    dev = torch.device("cuda", local if world > 1 else 0)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    s = Stream(wl.views, wl.frames, wl.tok_per_frame, wl.text_len, wl.H, wl.Hkv, wl.d, wl.rope_base)
+    for k in range(wl.steps + 1):  # the cache the drafted blocks are checked against
+        inp = window_inputs(wid, 0, k)
+        q = to_dev(inp["Q"])
+        s.insert(to_dev(inp["K"]), to_dev(inp["V"]))
+        s.attend(q, torch.empty(q.shape, dtype=torch.float32, device=dev))
+    sets = 4
+    blocks = [{x: to_dev(verify_inputs(wid, c)[x]) for x in ("Q", "K", "V")} for c in range(sets)]
+    nx = wl.verify_tokens
+    out = torch.empty((nx, wl.H, wl.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    clk = ClockSampler(gpu_id(dev))
+    clk.start()
+    for k in range(args.warmup):
+        b = blocks[k % sets]
+        s.attend_ext(b["Q"], b["K"], b["V"], out)
+    torch.cuda.synchronize()
+    launches0 = s.info().launches
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    clk.mark_start()
+    start.record(stream)
+    for k in range(args.steps):
+        b = blocks[k % sets]
+        s.attend_ext(b["Q"], b["K"], b["V"], out)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk.mark_end()
+    clk.stop()
+    barrier(world)
+    launches = s.info().launches - launches0
+    ms = max_over_ranks(start.elapsed_time(end), world) / args.steps
+    L = wl.window_len
+    fl = 4.0 * wl.d * wl.H * sum(L + t + 1 for t in range(nx))  # block token t sees L + t + 1 keys
+    # end to end: pinned host block in, result out, inside the timed region
+    pin = [{x: torch.from_numpy(np.ascontiguousarray(verify_inputs(wid, c)[x]).view(np.int16)).pin_memory()
+            for x in ("Q", "K", "V")} for c in range(sets)]
+    pin_out = torch.empty((nx, wl.H, wl.d), dtype=torch.float32).pin_memory()
+    dq, dk, dv = (torch.empty_like(blocks[0][x]) for x in ("Q", "K", "V"))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(args.steps, 64))
+    e0.record(stream)
+    for k in range(n_e2e):
+        hb = pin[k % sets]
+        dq.copy_(hb["Q"], non_blocking=True)
+        dk.copy_(hb["K"], non_blocking=True)
+        dv.copy_(hb["V"], non_blocking=True)
+        s.attend_ext(dq, dk, dv, out)
+        pin_out.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
+    s.close()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    h2d = int(dq.numel() + dk.numel() + dv.numel()) * 2
+    return {
+        "metric": METRIC,
+        "value": round(world * fl / (ms * 1e-3) / 1e12, 4),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "us_per_verify_call": round(ms * 1e3, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": f"verify: {nx}-token drafted blocks after the text of the medium window "
+                               f"(L = {L}, H{wl.H}/Hkv{wl.Hkv}/d{wl.d})", "workload_id": wid,
+                   "algorithmic_mflop_per_call": round(fl / 1e6, 2),
+                   "l2": "operands of one call fit in L2 (latency-bound shape)"},
+        "e2e": {"value": round(world * fl / (e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": int(out.numel()) * 4, "api": "Stream.attend_ext after pinned host copies"},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+
+
 def run_reference(args):
     """The oracle arm: the fp64 CPU oracle, as it stands, on host cores."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -488,6 +595,13 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         res = run_reference(args)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    from streaming_kv_cache_stream_b200.inputs import WORKLOADS as _W
+
+    if _W[args.workload].verify_calls:
+        res = run_verify(args)
         if res is not None:
             print(json.dumps(res), flush=True)
         return

@@ -161,3 +161,41 @@ def test_edge_shapes(shape):
         compare(from_dev(out), orc.verify(f64(bits["Q"]), f64(bits["K"]), f64(bits["V"])), f"{shape} verify {nx}")
     s.sync()
     s.close()
+
+
+def test_verify_interleaved_with_steps():
+    """Drafted blocks between window steps: a verify call leaves the window (and
+    the next attend of the same queries) unchanged, and the next step rotates
+    the whole window again. Medium window: prefill, step, verify, attend again,
+    step, verify, attend."""
+    import torch
+
+    wl = WORKLOADS[2]
+    s = make_stream(wl)
+    orc = make_oracle(wl)
+    for k in range(3):
+        inp = window_inputs(2, 0, k)
+        Q, K, V = (to_dev(inp[x]) for x in ("Q", "K", "V"))
+        out = out_like(Q)
+        s.insert(K, V)
+        s.attend(Q, out)
+        Qf, Kf, Vf = f64(inp["Q"]), f64(inp["K"]), f64(inp["V"])
+        want = orc.prefill(Qf, Kf, Vf) if k == 0 else orc.step(Qf, Kf, Vf)
+        torch.cuda.synchronize()
+        compare(from_dev(out), want, f"step {k}")
+        if k == 0:
+            continue
+        first = from_dev(out)
+        for call in range(2):
+            v = verify_inputs(5, 8 * k + call)
+            Qx, Kx, Vx = (to_dev(v[x]) for x in ("Q", "K", "V"))
+            ox = out_like(Qx)
+            s.attend_ext(Qx, Kx, Vx, ox)
+            torch.cuda.synchronize()
+            compare(from_dev(ox), orc.verify(f64(v["Q"]), f64(v["K"]), f64(v["V"])), f"verify after step {k}")
+        again = out_like(Q)
+        s.attend(Q, again)
+        torch.cuda.synchronize()
+        assert np.array_equal(from_dev(again), first), "a drafted block changed the next attend of the same queries"
+    s.sync()
+    check_cache_bitexact(s, orc, wl)
