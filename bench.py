@@ -170,21 +170,29 @@ def gpu_id(dev):
         return str(dev.index or 0)
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """Rank, world and local rank from the torchrun environment; joins the
+    process group when world > 1 (NCCL on GPUs; gloo when CUDA is absent, which
+    the CPU tests use). Returns (world, rank, local)."""
     import torch
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    cuda = torch.cuda.is_available()
+    backend = backend or ("nccl" if cuda else "gloo")
     if world > 1:
         import datetime
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif cuda:
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -196,18 +204,28 @@ def barrier(world):
         import torch.distributed as dist
 
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(x, world):
+    """The largest of every rank's x (every rank gets it): device times are
+    reported as the slowest rank's."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tflops(flops_per_rank, ms, world):
+    """Whole-job throughput of weak-scaling replicas: every rank did
+    flops_per_rank in (at most) ms, the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
 
 
 # ----------------------------------------------------------- CPU oracle leg
@@ -319,7 +337,7 @@ def run_ours(args):
 
     fl_layer = step_flops(wl)
     ms_per_step = elapsed_ms / args.steps
-    value = world * fl_layer * layers / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(fl_layer * layers, ms_per_step, world)
     att_avg_ms = statistics.mean(att_ms)
     att_tflops = fl_layer / (att_avg_ms * 1e-3) / 1e12
     # kv_stream_insert moves, per kv head: the step's new K/V rows (read from the
