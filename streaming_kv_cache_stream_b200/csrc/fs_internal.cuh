@@ -2,6 +2,8 @@
 // kernels, and the position arithmetic of the view-major window.
 #pragma once
 #include <cstdint>
+#include <cstdlib>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -94,6 +96,34 @@ struct InsertParams {
     uint16_t* Kl;           // fp16 rotated key, lo part
     uint16_t* V16;          // fp16 V
 };
+
+// Launches `kernel` with programmatic stream serialisation: its launch and set-up
+// may overlap the end of the previous kernel on the stream; the kernel itself
+// calls grid_dependency_wait() before touching memory that kernel may use.
+// FS_PDL=0 in the environment turns the overlap off (ordinary stream order).
+inline bool overlapped_launch_enabled() {
+    static const bool on = [] {
+        const char* e = std::getenv("FS_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = overlapped_launch_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Launchers (defined in the .cu files); all enqueue on `stream` and return the
 // launch's cudaError_t.

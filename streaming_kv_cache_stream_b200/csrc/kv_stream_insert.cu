@@ -65,6 +65,8 @@ __device__ __forceinline__ int source_token(const InsertParams& p, int row) {
 
 template <int D>
 __global__ void __launch_bounds__(kInsertThreads) kv_stream_insert_kernel(const InsertParams p) {
+    grid_dependency_wait();     // the previous kernel (say, an attention reading these operands) is done
+    allow_dependents_launch();  // the next kernel may start its set-up
     constexpr int kPairs = D / 16;  // threads per (row, kv head)
     const unsigned gid = blockIdx.x * kInsertThreads + threadIdx.x;
     const unsigned nrows = unsigned(p.row_end - p.row_begin);
@@ -129,8 +131,7 @@ template <int D>
 cudaError_t launch_d(const InsertParams& p, cudaStream_t stream) {
     const long long threads = (long long)(p.row_end - p.row_begin) * p.Hkv * (D / 16);
     const unsigned blocks = unsigned((threads + kInsertThreads - 1) / kInsertThreads);
-    kv_stream_insert_kernel<D><<<blocks, kInsertThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_overlapped(kv_stream_insert_kernel<D>, dim3(blocks), dim3(kInsertThreads), 0, stream, p);
 }
 
 }  // namespace

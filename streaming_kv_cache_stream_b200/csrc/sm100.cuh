@@ -74,6 +74,16 @@ struct BoundedWait {
     }
 };
 
+// ------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while the
+// previous kernel on the stream finishes. grid_dependency_wait() returns once
+// that kernel has completed and its memory is visible (immediately when it was
+// not launched that way); every thread calls it before touching global memory
+// an earlier kernel may write or read. allow_dependents_launch() lets the next
+// such kernel start launching (it still waits for this one to complete).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ------------------------------------------------------------------- fences
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -265,6 +265,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             return;
         }
     }
+    grid_dependency_wait();     // the insert that wrote this call's operands is done
+    allow_dependents_launch();  // the next kernel may start its set-up
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -792,8 +794,7 @@ cudaError_t launch_d(const AttnParams& p, const CUtensorMap& tq, const CUtensorM
     }
     const int units = (p.q_tiles + 3) / 4;
     const unsigned grid = unsigned(2 * units * p.Hkv * p.splits);
-    stream_attn_kernel<D><<<grid, kThreads, smem, stream>>>(p, tq, tkh, tkl, tv16);
-    return cudaGetLastError();
+    return launch_overlapped(stream_attn_kernel<D>, dim3(grid), dim3(kThreads), smem, stream, p, tq, tkh, tkl, tv16);
 }
 
 }  // namespace
