@@ -15,16 +15,24 @@
 // of operands per 512 query rows: on B200 the tensor pipes of all SMs would
 // otherwise need more from L2 than it delivers. A query tile packs 128/G
 // tokens x the G query heads of one kv group (GQA). The keys were rotated for
-// this step by kv_stream_rope (at their shifted positions, as fp16 hi + lo; V
-// as fp16); this kernel rotates its query rows.
+// this step by kv_stream_insert (at their shifted positions, as fp16 hi + lo;
+// V as fp16); this kernel rotates its query rows.
 //
 // Warp roles per CTA (12 warps):
+//   warps 0-3   prologue: classify the key tiles against the unit's and each
+//               group's query range; then
 //   warp 0      TMA producer: this CTA's halves of K hi/lo and V, 2 + 2 stages;
 //   warp 1      TMEM allocation; in the even CTA, the single MMA issuer;
-//   warps 4-7   group a: RoPE of its query rows, then its online softmax;
-//   warps 8-11  group b: the same.
+//   warps 4-11  prologue: RoPE of the query rows (group a: 4-7, group b: 8-11)
+//               from a TMA-loaded bf16 tile, in place in shared memory; then
+//               the online softmax of every S tile of both groups, warpgroup w
+//               on key columns [64 w, 64 w + 64); then the epilogue, warpgroup
+//               w finishing group w.
 // TMEM per CTA: S_a, S_b (fp32 scores, 128 columns each; P as fp16 over the
 // first 64 columns of its S) and O_a, O_b (fp32, D columns each).
+// The kernel is launched with programmatic stream serialisation: it waits for
+// the previous kernel on the stream (the insert that wrote its operands) at
+// entry, and lets the next one start launching.
 // MMA issue order for key tile k: QK_a(k), PV_b(k-1), QK_b(k), PV_a(k). A QK
 // into S_g waits for the previous PV_g (it reads P_g from the same columns),
 // and that wait always has other work queued on the tensor pipe; while one
