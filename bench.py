@@ -54,6 +54,12 @@ def step_flops(wl):
     return 4.0 * wl.d * wl.H * visible_pairs_step(wl.views, wl.frames, wl.tok_per_frame, wl.text_len)
 
 
+def verify_flops(wl):
+    """Algorithmic FLOPs of one drafted-block verify call: block token t sees the
+    L window keys and block tokens 0..t."""
+    return 4.0 * wl.d * wl.H * sum(wl.window_len + t + 1 for t in range(wl.verify_tokens))
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -508,7 +514,7 @@ def run_verify(args):
     launches = s.info().launches - launches0
     ms = max_over_ranks(start.elapsed_time(end), world) / args.steps
     L = wl.window_len
-    fl = 4.0 * wl.d * wl.H * sum(L + t + 1 for t in range(nx))  # block token t sees L + t + 1 keys
+    fl = verify_flops(wl)
     # end to end: pinned host block in, result out, inside the timed region
     pin = [{x: torch.from_numpy(np.ascontiguousarray(verify_inputs(wid, c)[x]).view(np.int16)).pin_memory()
             for x in ("Q", "K", "V")} for c in range(sets)]
