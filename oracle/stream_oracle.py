@@ -27,6 +27,10 @@ What it computes, and where the pages define it (FlashDrive, arXiv 2608.12932):
 * Speculative verification of a drafted 8-token block in one forward --
   FlashDrive README (z-lab/flashdrive), "Speculative reasoning (DFlash)";
   technical summary (gist.science), Methodology 2.
+* Accepted draft tokens become context for the next drafted block (the
+  decode stage produces reasoning tokens after the prompt; the drafter's
+  blocks of 8 are accepted 5.6 tokens at a time on average) -- technical
+  summary (gist.science), Methodology 2, "Efficiency".
 
 The pages fix no RoPE variant, base, mask formula or head grouping. The
 readings used here (each one also listed in the design notes):
@@ -41,8 +45,11 @@ readings used here (each one also listed in the design notes):
   the queries of every step.
 * Query head h reads kv head h // (H / Hkv) (contiguous grouping).
 * Softmax scale 1/sqrt(d); no soft-capping, no sinks.
-* The verify block's n_x tokens sit at positions L .. L + n_x - 1, see the
-  whole window plus, causally, each other, and are not kept in the cache.
+* Accepted tokens are appended to a decode tail right after the text (tail
+  token j at position L + j); a verify block's n_x tokens sit after the tail,
+  at L + tail .. L + tail + n_x - 1, see the whole window, the tail and,
+  causally, each other, and are not kept. A window step starts a new window
+  and with it an empty tail (a new prompt, a new reasoning pass).
 
 Data structure: a deque of frames per view, with an insertion counter as the
 frame id. This is deliberately not a ring buffer, so it shares no index
@@ -203,6 +210,8 @@ class ViewMajorWindow:
         self.text_V = None
         self.next_id = [0] * views
         self.filled = False
+        self.tail_K: list = []  # accepted decode tokens after the text, oldest first
+        self.tail_V: list = []
 
     @property
     def window_len(self) -> int:
@@ -229,6 +238,7 @@ class ViewMajorWindow:
                 self._push(v, K[a:a + self.n], V[a:a + self.n])
         t0 = self.V * self.T * self.n
         self.text_K, self.text_V = K[t0:].copy(), V[t0:].copy()
+        self.tail_K, self.tail_V = [], []
         self.filled = True
 
     def step(self, K_new: np.ndarray, V_new: np.ndarray) -> None:
@@ -243,6 +253,26 @@ class ViewMajorWindow:
             self.views[v].popleft()
         t0 = self.V * self.n
         self.text_K, self.text_V = K_new[t0:].copy(), V_new[t0:].copy()
+        self.tail_K, self.tail_V = [], []
+
+    def append(self, K_acc: np.ndarray, V_acc: np.ndarray) -> None:
+        """Accepted decode tokens [n, Hkv, d], appended after the text (and the earlier tail)."""
+        if not self.filled:
+            raise ValueError("append before prefill")
+        for i in range(K_acc.shape[0]):
+            self.tail_K.append(np.array(K_acc[i], dtype=np.float64))
+            self.tail_V.append(np.array(V_acc[i], dtype=np.float64))
+
+    @property
+    def tail_len(self) -> int:
+        return len(self.tail_K)
+
+    def materialise_tail(self, Hkv: int, d: int):
+        """Tail K, V [tail, Hkv, d] (empty arrays when there is none)."""
+        if not self.tail_K:
+            z = np.zeros((0, Hkv, d))
+            return z, z.copy()
+        return np.stack(self.tail_K), np.stack(self.tail_V)
 
     def materialise(self):
         """Window K, V [L, Hkv, d] in view-major order, plus per-row bookkeeping.
@@ -289,7 +319,9 @@ class StreamOracle:
 
     ``prefill`` is the stream's first call (whole window, full causal over the
     view-major sequence); ``step`` is a window step (new frame per view plus
-    text); ``verify`` appends a drafted block after the text without keeping it.
+    text); ``append`` persists accepted decode tokens after the text;
+    ``verify`` attends a drafted block after the text and the tail without
+    keeping it.
     Inputs are float64 arrays (use ``bf16_bits_to_f64`` on the shared bf16
     bytes). ``rows`` restricts the computed queries to a subset of query
     indices, so full-size cases can be checked on samples.
@@ -319,23 +351,37 @@ class StreamOracle:
         return self._attend(Q, self.win.step_query_positions(), rows, Kw, Vw,
                             self.win.key_positions())
 
+    def append(self, K_acc, V_acc):
+        """Persist accepted decode tokens after the text (see ViewMajorWindow.append)."""
+        self.win.append(K_acc, V_acc)
+
     def verify(self, Q_x, K_x, V_x, rows=None):
-        """A drafted block of n_x tokens at positions L .. L+n_x-1, not persisted."""
+        """A drafted block of n_x tokens right after the text and the decode
+        tail (positions L + tail .. L + tail + n_x - 1), not persisted."""
         Kw, Vw, *_ = self.win.materialise()
+        Kt, Vt = self.win.materialise_tail(self.Hkv, self.d)
         L = self.win.window_len
+        t = Kt.shape[0]
         nx = Q_x.shape[0]
-        K = np.concatenate([Kw, K_x], axis=0)
-        V = np.concatenate([Vw, V_x], axis=0)
-        kpos = np.arange(L + nx, dtype=np.int64)
-        qpos = np.arange(L, L + nx, dtype=np.int64)
+        K = np.concatenate([Kw, Kt, K_x], axis=0)
+        V = np.concatenate([Vw, Vt, V_x], axis=0)
+        kpos = np.arange(L + t + nx, dtype=np.int64)
+        qpos = np.arange(L + t, L + t + nx, dtype=np.int64)
         return self._attend(Q_x, qpos, rows, K, V, kpos)
 
     def cache_rows(self):
         """Pre-RoPE cached rows with their (view, frame_id, token, position).
 
         Used for the bit-exact comparison with the device cache: rows match by
-        (view, frame_id, token) for frames and by text index for text.
+        (view, frame_id, token) for frames, by text index for text (view -1)
+        and by tail index for the decode tail (view -2).
         """
         Kw, Vw, view, fid, tok = self.win.materialise()
-        return dict(K=Kw, V=Vw, view=view, frame_id=fid, token=tok,
-                    pos=self.win.key_positions())
+        Kt, Vt = self.win.materialise_tail(self.Hkv, self.d)
+        t = Kt.shape[0]
+        L = self.win.window_len
+        return dict(K=np.concatenate([Kw, Kt]), V=np.concatenate([Vw, Vt]),
+                    view=np.concatenate([view, np.full(t, -2)]),
+                    frame_id=np.concatenate([fid, np.full(t, -1)]),
+                    token=np.concatenate([tok, np.arange(t)]),
+                    pos=np.arange(L + t, dtype=np.int64))

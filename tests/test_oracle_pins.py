@@ -155,6 +155,10 @@ class _History:
             self.frames[v].append((K[v * self.n:(v + 1) * self.n], V[v * self.n:(v + 1) * self.n]))
         t = self.V * self.n
         self.text = (K[t:], V[t:])
+        self.tail = []
+
+    def append(self, K, V):
+        self.tail = getattr(self, "tail", []) + [(K[i], V[i]) for i in range(K.shape[0])]
 
     def window(self):
         toks = []
@@ -234,8 +238,71 @@ def pin_brute_force(shape, steps=3, seed=5):
         np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
 
 
+def pin_brute_force_decode_tail(shape, seed=9):
+    """Drafted blocks verified against window + accepted tail, rebuilt from the
+    full history with scalar loops: tail tokens follow the text, a block follows
+    the tail, and a window step empties the tail."""
+    rng = np.random.default_rng(seed)
+    V, T, n, X, H, Hkv, d = (shape[k] for k in ("views", "frames", "tok_per_frame", "text_len", "H", "Hkv", "d"))
+    L = V * T * n + X
+    N = V * n + X
+    orc = StreamOracle(V, T, n, X, H, Hkv, d)
+    hist = _History(**shape)
+
+    def draw(m, heads):
+        return bf16_bits_to_f64(_rand(rng, m, heads, d))
+
+    K, Vv = draw(L, Hkv), draw(L, Hkv)
+    orc.prefill(draw(L, H), K, Vv)
+    hist.prefill(K, Vv)
+    hist.tail = []
+    for rnd in range(2):
+        for n_acc, n_x in ((3, 2), (2, 3)):
+            Qx, Kx, Vx = draw(n_x, H), draw(n_x, Hkv), draw(n_x, Hkv)
+            got = orc.verify(Qx, Kx, Vx)
+            toks = hist.window() + hist.tail + [(Kx[i], Vx[i]) for i in range(n_x)]
+            t = len(hist.tail)
+            want = _brute_attend(list(Qx), [L + t + j for j in range(n_x)], toks, H, Hkv, d)
+            np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+            Ka, Va = draw(n_acc, Hkv), draw(n_acc, Hkv)
+            orc.append(Ka, Va)
+            hist.append(Ka, Va)
+        # a window step: new frames, new text, no tail
+        K, Vv = draw(N, Hkv), draw(N, Hkv)
+        orc.step(draw(N, H), K, Vv)
+        hist.step(K, Vv)
+
+
 def test_brute_force_tiny():
     pin_brute_force(TINY, steps=3)
+
+
+def test_brute_force_decode_tail():
+    pin_brute_force_decode_tail(TINY)
+    pin_brute_force_decode_tail(TINY_G, seed=10)
+
+
+def test_append_then_verify_equals_longer_block():
+    """Appending accepted tokens, then verifying a block, gives the block's rows
+    of one verify over (accepted ++ block): the tail sits exactly where the
+    accepted tokens sat in the longer block."""
+    wl = WORKLOADS[1]
+    rng = np.random.default_rng(12)
+    a = StreamOracle(wl.views, wl.frames, wl.tok_per_frame, wl.text_len, wl.H, wl.Hkv, wl.d)
+    b = StreamOracle(wl.views, wl.frames, wl.tok_per_frame, wl.text_len, wl.H, wl.Hkv, wl.d)
+    inp = window_inputs(1, 0, 0)
+    f = [bf16_bits_to_f64(inp[k]) for k in ("Q", "K", "V")]
+    a.prefill(*f)
+    b.prefill(*f)
+    n_acc, nx = 5, 8
+    Q = bf16_bits_to_f64(_rand(rng, n_acc + nx, wl.H, wl.d))
+    K = bf16_bits_to_f64(_rand(rng, n_acc + nx, wl.Hkv, wl.d))
+    Vv = bf16_bits_to_f64(_rand(rng, n_acc + nx, wl.Hkv, wl.d))
+    long = a.verify(Q, K, Vv)
+    b.append(K[:n_acc], Vv[:n_acc])
+    short = b.verify(Q[n_acc:], K[n_acc:], Vv[n_acc:])
+    np.testing.assert_allclose(short, long[n_acc:], rtol=0, atol=1e-13)
+    assert b.cache_rows()["K"].shape[0] == wl.window_len + n_acc
 
 
 def test_brute_force_tiny_gqa():
@@ -526,3 +593,31 @@ def test_planted_no_eviction(monkeypatch):
         t0 = self.V * self.n
         self.text_K, self.text_V = K_new[t0:].copy(), V_new[t0:].copy()
     _expect_caught(monkeypatch, (ViewMajorWindow, "step"), bad, ALL_PINS)
+
+
+TAIL_PINS = [lambda: pin_brute_force_decode_tail(TINY), lambda: pin_brute_force_decode_tail(TINY_G, seed=10)]
+
+
+def test_planted_tail_before_text(monkeypatch):
+    """A tail spliced in before the text (wrong positions) is caught."""
+    def bad(self, Q_x, K_x, V_x, rows=None):
+        Kw, Vw, *_ = self.win.materialise()
+        Kt, Vt = self.win.materialise_tail(self.Hkv, self.d)
+        X = self.win.X
+        K = np.concatenate([Kw[:len(Kw) - X], Kt, Kw[len(Kw) - X:], K_x])
+        V = np.concatenate([Vw[:len(Vw) - X], Vt, Vw[len(Vw) - X:], V_x])
+        n = K.shape[0]
+        nx = Q_x.shape[0]
+        return self._attend(Q_x, np.arange(n - nx, n), rows, K, V, np.arange(n))
+    _expect_caught(monkeypatch, (StreamOracle, "verify"), bad, TAIL_PINS)
+
+
+def test_planted_tail_kept_across_steps(monkeypatch):
+    """A tail that survives a window step is caught."""
+    orig = ViewMajorWindow.step
+
+    def bad(self, K_new, V_new):
+        keep = (self.tail_K, self.tail_V)
+        orig(self, K_new, V_new)
+        self.tail_K, self.tail_V = keep
+    _expect_caught(monkeypatch, (ViewMajorWindow, "step"), bad, TAIL_PINS)
