@@ -36,6 +36,18 @@
  *     last failure is available from fs_stream_last_error (per handle) or
  *     fs_last_error (calling thread, for failures without a handle).
  *   - A handle is not thread-safe: one host thread at a time per handle.
+ *   - Supported input range. The tensor-core operands are fp16 (11-bit
+ *     significands, largest finite value 65504): V as fp16; each rotated key
+ *     element as an fp16 hi + lo pair; each rotated query element, scaled by
+ *     log2(e)/sqrt(d), as an fp16 hi + lo pair. Rotation mixes the pair
+ *     (i, i+d/2), so a rotated element is at most sqrt(2) times the larger of
+ *     the two. Inputs are therefore supported when they are finite and
+ *       |V| <= 65504,  |K| <= 46318 (65504/sqrt(2)),
+ *       |Q| <= 46318 * sqrt(d) / log2(e)  (363,000 at d = 128; 256,000 at d = 64).
+ *     The kernels check every converted element; one out of range (or NaN)
+ *     sets a flag that the next fs_stream_sync or fs_stream_debug_export
+ *     reports as FS_ERR_RANGE (the outputs since the previous check are then
+ *     not valid; the flag is cleared).
  */
 #ifndef FS_STREAM_H
 #define FS_STREAM_H
@@ -52,6 +64,7 @@ extern "C" {
 #define FS_ERR_CUDA            -3 /* a CUDA runtime/driver call failed (message has it)    */
 #define FS_ERR_DEVICE_TIMEOUT  -4 /* a bounded device-side wait gave up (no hang)          */
 #define FS_ERR_OOM             -5 /* device or host allocation failed                       */
+#define FS_ERR_RANGE           -6 /* an input exceeded the supported range (see below)      */
 
 /* Stream states. */
 #define FS_STATE_EXPECT_PREFILL 0 /* after create/reset: insert takes the whole window     */
@@ -60,6 +73,8 @@ extern "C" {
 
 /* Largest drafted block fs_stream_attend_ext accepts. */
 #define FS_MAX_VERIFY_TOKENS 256
+/* Largest persisted decode tail (accepted tokens after the text, fs_stream_append). */
+#define FS_MAX_TAIL_TOKENS 1024
 
 typedef struct fs_stream* fs_stream_t;
 
@@ -73,23 +88,34 @@ typedef struct fs_stream_info_t {
     int query_tokens;    /* queries the next fs_stream_attend expects (0: none allowed)  */
     int head;            /* ring slot holding each view's oldest frame                   */
     long long steps;     /* window steps inserted since the prefill                      */
-    long long cache_bytes; /* device bytes owned by the handle                           */
+    long long cache_bytes; /* device bytes owned by the handle (the shared RoPE table aside) */
     long long launches;  /* kernels this handle has launched since create                 */
+    int tail_tokens;     /* persisted decode-tail tokens after the text (fs_stream_append)  */
+    int rebase_every;    /* R: every R-th window step re-rotates the whole window           */
 } fs_stream_info_t;
 
 /*
  * fs_stream_create -- allocate one layer's static KV cache (FlashDrive README,
- * "System optimizations": static KV cache) and its RoPE table on the current
- * CUDA device.
+ * "System optimizations": static KV cache) on the current CUDA device.
  *   views, frames, tok_per_frame >= 1; text_len >= 0; H, Hkv >= 1 with H % Hkv == 0
  *   and 128 % (H/Hkv) == 0; d in {64, 128}; rope_base > 0 (10000 in the
- *   synthetic workloads). L + FS_MAX_VERIFY_TOKENS must be <= 262144 (2048 key tiles
- *   of 128 rows per kv head).
+ *   synthetic workloads). L + FS_MAX_TAIL_TOKENS + FS_MAX_VERIFY_TOKENS must be
+ *   <= 262144 (2048 key tiles of 128 rows per kv head).
  * Device layout of the cache (owned by the handle, zero-initialised):
- *   K_cache, V_cache [Hkv][R][d] bf16 with R = L + FS_MAX_VERIFY_TOKENS rows per
- *   kv head: rows [0, views*frames*tok_per_frame) are the per-view rings
- *   (view v, slot s, token i at row (v*frames + s)*tok_per_frame + i), then
- *   text_len text rows, then scratch rows for a drafted block.
+ *   K_cache, V_cache [Hkv][R][d] bf16 with R = L + FS_MAX_TAIL_TOKENS +
+ *   FS_MAX_VERIFY_TOKENS rows per kv head: rows [0, views*frames*tok_per_frame)
+ *   are the per-view rings (view v, slot s, token i at row
+ *   (v*frames + s)*tok_per_frame + i), then text_len text rows, then the
+ *   persisted decode tail, then scratch rows for a drafted block.
+ *   Next to it the handle keeps the attention operands (each key rotated once,
+ *   as fp16 hi + lo, and V as fp16, same layout), a device-resident ring state
+ *   (head slot and step count, advanced by the insert kernel) and split-KV
+ *   scratch. The cos/sin table is shared by handles of the same device, d,
+ *   rope_base and size.
+ * Keys are rotated once, when they enter the cache, at angle index p + k*n
+ * (p: window position, k: window steps since the last re-base); queries at
+ * their position + k*n. Every R-th window step (R = 16, or FS_REBASE_STEPS in
+ * the environment at create, 1..4096) re-rotates the whole window at k = 0.
  * On success *out receives the handle and the state is FS_STATE_EXPECT_PREFILL.
  * Errors: FS_ERR_ARG, FS_ERR_OOM, FS_ERR_CUDA (nothing is leaked).
  */
@@ -124,6 +150,18 @@ int fs_stream_reset(fs_stream_t s);
 int fs_stream_insert(fs_stream_t s, const void* K_new, const void* V_new);
 
 /*
+ * fs_stream_insert_batch -- fs_stream_insert for n layers in one kernel launch
+ * (FlashDrive README, "System optimizations": static KV cache; one launch per
+ * window step instead of one per layer). handles[i] receives K_new[i] and
+ * V_new[i] (device pointers, sizes as for fs_stream_insert). All handles must
+ * share the window shape, Hkv, d, rope_base, device and stream (handles[0]'s
+ * stream runs the launch), be distinct, and be all in EXPECT_PREFILL or all
+ * past it. Each layer's device ring state advances as in fs_stream_insert.
+ * Errors: FS_ERR_ARG (nothing enqueued), FS_ERR_STATE, FS_ERR_CUDA.
+ */
+int fs_stream_insert_batch(fs_stream_t* handles, int n, const void* const* K_new, const void* const* V_new);
+
+/*
  * fs_stream_attend -- attention of the last inserted tokens (kernel stream_attn).
  *   State PREFILLED: Q and out are [L][H][d]; query t sits at position t
  *     (plain causal attention over the view-major window).
@@ -141,10 +179,24 @@ int fs_stream_insert(fs_stream_t s, const void* K_new, const void* V_new);
 int fs_stream_attend(fs_stream_t s, const void* Q, void* out);
 
 /*
+ * fs_stream_append -- persist n_acc accepted tokens (pre-RoPE K/V, [n_acc][Hkv][d]
+ * bf16, device) at the end of the decode tail: the tokens a verified drafted
+ * block contributed (FlashDrive README, "Speculative reasoning (DFlash)";
+ * technical summary, Methodology 2: blocks of 8 drafted tokens, 5.6 accepted on
+ * average). Tail token j sits at position L + j, after the text; every later
+ * drafted block sees it. The next window insert (fs_stream_insert or
+ * fs_stream_insert_batch) empties the tail: a new window starts a new
+ * reasoning pass. tail + n_acc <= FS_MAX_TAIL_TOKENS.
+ * State: PREFILLED or STREAMING. Errors: FS_ERR_ARG, FS_ERR_STATE, FS_ERR_CUDA.
+ */
+int fs_stream_append(fs_stream_t s, const void* K_acc, const void* V_acc, int n_acc);
+
+/*
  * fs_stream_attend_ext -- verify a drafted block of n_x tokens in one forward
  * (FlashDrive README, "Speculative reasoning (DFlash)"; technical summary,
- * Methodology 2). The block's tokens sit at positions L .. L+n_x-1, after the
- * text; each sees the whole cached window plus, causally, the block.
+ * Methodology 2). The block's tokens sit at positions L + tail .. L + tail +
+ * n_x - 1, after the text and the persisted decode tail; each sees the whole
+ * cached window, the tail and, causally, the block.
  *   Q_x [n_x][H][d] bf16, out [n_x][H][d] fp32; K_x, V_x [n_x][Hkv][d] bf16
  *   (pre-RoPE); 1 <= n_x <=
  *   FS_MAX_VERIFY_TOKENS. The block's K/V go to the handle's scratch rows and are
@@ -183,21 +235,25 @@ int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x,
 /*
  * fs_stream_step_host -- one insert + attend with HOST buffers: copies K_new,
  * V_new and Q (bf16) to the device (staging buffers owned by the handle), runs
- * fs_stream_insert and fs_stream_attend, and copies out back, all enqueued on
- * the handle's stream. Sizes follow the current state exactly as for
- * fs_stream_insert / fs_stream_attend; out_h receives fp32. The staging
- * buffers are allocated on the first call (and grown if a later call needs
- * more), so make the first call outside any stream capture. With pinned host
- * memory the call is
- * asynchronous; the caller synchronises (fs_stream_sync) before reading out_h.
+ * fs_stream_insert and fs_stream_attend on the handle's stream, and copies out
+ * back. The uploads run on a copy stream of the handle (after the previous
+ * call's kernels have read the staging buffer) and the download on a second
+ * one, so consecutive calls on different handles overlap uploads, kernels and
+ * downloads. Sizes follow the current state exactly as for fs_stream_insert /
+ * fs_stream_attend; out_h receives fp32. The staging buffers and copy streams
+ * are created on the first call (buffers grown if a later call needs more), so
+ * make the first call outside any stream capture. With pinned host memory the
+ * call is asynchronous; out_h is complete once fs_stream_sync(s) returns.
  * Errors: as fs_stream_insert and fs_stream_attend.
  */
 int fs_stream_step_host(fs_stream_t s, const void* K_new_h, const void* V_new_h,
                         const void* Q_h, void* out_h);
 
-/* Block until the handle's enqueued work is done. Returns FS_ERR_DEVICE_TIMEOUT if a
- * kernel of this handle gave up on a bounded wait since the last check (the flag is
- * cleared), FS_ERR_CUDA on an asynchronous CUDA error. */
+/* Block until the handle's enqueued work (its stream and host-path copy streams)
+ * is done. Returns FS_ERR_DEVICE_TIMEOUT if a kernel of this handle gave up on a
+ * bounded wait since the last check, FS_ERR_RANGE if an input was outside the
+ * supported range (see the conventions above; the flags are cleared), FS_ERR_CUDA
+ * on an asynchronous CUDA error. */
 int fs_stream_sync(fs_stream_t s);
 
 /* Sizes and state. */
@@ -206,12 +262,13 @@ int fs_stream_info(fs_stream_t s, fs_stream_info_t* info);
 /*
  * fs_stream_debug_export -- synchronous copy of the physical cache to HOST
  * buffers for tests: K_phys, V_phys [Hkv][rows][d] bf16 with rows =
- * views*frames*tok_per_frame + text_len (ring rows then text rows, the device
- * layout above), pos_phys[rows] = each row's current window position as the
- * attention kernel computes it, frame_id_phys[rows] = the insertion counter of
+ * views*frames*tok_per_frame + text_len + tail_tokens (ring rows, text rows,
+ * decode-tail rows: the device layout above), pos_phys[rows] = each row's
+ * current window position as the attention kernel computes it (from the
+ * device-resident ring head), frame_id_phys[rows] = the insertion counter of
  * the frame a ring row belongs to (frames of the prefill are 0..frames-1, the
- * k-th step inserts frame frames-1+k; -1 for text rows). Any pointer may be
- * NULL to skip that output. State: not EXPECT_PREFILL.
+ * k-th step inserts frame frames-1+k; -1 for text and tail rows). Any pointer
+ * may be NULL to skip that output. State: not EXPECT_PREFILL.
  */
 int fs_stream_debug_export(fs_stream_t s, void* K_phys, void* V_phys,
                            int32_t* pos_phys, int32_t* frame_id_phys);

@@ -19,10 +19,12 @@ FS_ERR_STATE = -2
 FS_ERR_CUDA = -3
 FS_ERR_DEVICE_TIMEOUT = -4
 FS_ERR_OOM = -5
+FS_ERR_RANGE = -6
 FS_STATE_EXPECT_PREFILL = 0
 FS_STATE_PREFILLED = 1
 FS_STATE_STREAMING = 2
 FS_MAX_VERIFY_TOKENS = 256
+FS_MAX_TAIL_TOKENS = 1024
 
 # Every symbol the header declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -33,7 +35,8 @@ class fs_stream_info_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "views", "frames", "tok_per_frame", "text_len", "H", "Hkv", "d", "window_len", "step_tokens",
         "state", "insert_tokens", "query_tokens", "head")] + [
-        ("steps", ctypes.c_longlong), ("cache_bytes", ctypes.c_longlong), ("launches", ctypes.c_longlong)]
+        ("steps", ctypes.c_longlong), ("cache_bytes", ctypes.c_longlong), ("launches", ctypes.c_longlong),
+        ("tail_tokens", ctypes.c_int), ("rebase_every", ctypes.c_int)]
 
 
 SIGNATURES = {
@@ -42,6 +45,8 @@ SIGNATURES = {
     "fs_stream_set_stream": (_I, [_P, _P]),
     "fs_stream_reset": (_I, [_P]),
     "fs_stream_insert": (_I, [_P, _P, _P]),
+    "fs_stream_insert_batch": (_I, [ctypes.POINTER(_P), _I, ctypes.POINTER(_P), ctypes.POINTER(_P)]),
+    "fs_stream_append": (_I, [_P, _P, _P, _I]),
     "fs_stream_attend": (_I, [_P, _P, _P]),
     "fs_stream_attend_ext": (_I, [_P, _P, _P, _P, _I, _P]),
     "fs_stream_attend_ext_static": (_I, [_P, _P, _P, _P, _I, _P]),
@@ -146,6 +151,11 @@ class Stream:
         self._bind_stream()
         _check(self._lib.fs_stream_insert(self.handle, _ptr(K_new), _ptr(V_new)), self.handle)
 
+    def append(self, K_acc, V_acc):
+        """Persist accepted tokens [n, Hkv, d] bf16 at the end of the decode tail."""
+        self._bind_stream()
+        _check(self._lib.fs_stream_append(self.handle, _ptr(K_acc), _ptr(V_acc), int(K_acc.shape[0])), self.handle)
+
     def attend(self, Q, out):
         """Q bf16 [tokens, H, d] -> out fp32 [tokens, H, d]."""
         self._bind_stream()
@@ -181,7 +191,7 @@ class Stream:
         import numpy as np
 
         i = self.info()
-        rows = i.window_len
+        rows = i.window_len + i.tail_tokens
         K = np.empty((self.Hkv, rows, self.d), dtype=np.uint16)
         V = np.empty_like(K)
         pos = np.empty(rows, dtype=np.int32)
@@ -191,3 +201,21 @@ class Stream:
             pos.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), fid.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))),
             self.handle)
         return dict(K=K, V=V, pos=pos, frame_id=fid)
+
+
+def insert_batch(streams, K_list, V_list):
+    """fs_stream_insert_batch: one kv_stream_insert launch for every layer's
+    handle (streams[i] gets K_list[i], V_list[i]); torch's current stream."""
+    import torch
+
+    n = len(streams)
+    if not (n == len(K_list) == len(V_list)) or n == 0:
+        raise ValueError("need one K and one V per stream")
+    lib = load()
+    cur = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for s in streams:
+        _check(lib.fs_stream_set_stream(s.handle, cur), s.handle)
+    hs = (_P * n)(*[s.handle.value for s in streams])
+    ks = (_P * n)(*[_ptr(k).value for k in K_list])
+    vs = (_P * n)(*[_ptr(v).value for v in V_list])
+    _check(lib.fs_stream_insert_batch(hs, n, ks, vs), streams[0].handle)

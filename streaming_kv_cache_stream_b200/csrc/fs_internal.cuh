@@ -12,8 +12,12 @@ namespace fs {
 constexpr int kTileRows = 128;          // query rows (token x head) and keys per tile
 constexpr int kMaxKeyTiles = 2048;      // key rows per kv head <= 2048 * 128
 constexpr int kMaxVerify = 256;         // scratch rows for a drafted block (FS_MAX_VERIFY_TOKENS)
+constexpr int kMaxTail = 1024;          // persisted decode-tail rows (FS_MAX_TAIL_TOKENS)
+constexpr int kMaxInsertBatch = 40;     // layers one kv_stream_insert launch covers
 constexpr unsigned kErrTimeout = 1u;    // device error word bits
 constexpr unsigned kErrBadLaunch = 2u;
+constexpr unsigned kErrRange = 4u;      // an fp16 operand would overflow (|x| > 65504) or is NaN
+constexpr float kF16Max = 65504.f;
 
 enum QueryMode : int { kQueryPrefill = 0, kQueryStep = 1, kQueryVerify = 2 };
 
@@ -22,7 +26,34 @@ struct WindowShape {
     int V, T, n, X;     // views, frames per view, tokens per frame, text tokens
     int ring_rows;      // V * T * n
     int head;           // ring slot holding every view's oldest frame
+    int tail;           // persisted decode-tail tokens after the text
 };
+
+// Ring state kept in device memory, one per handle. kv_stream_insert advances
+// it (the last block of the launch writes the new values); every kernel reads
+// it after its grid-dependency wait, so no launch parameter changes from one
+// window step to the next.
+//   head: ring slot holding each view's oldest frame;
+//   k:    window steps since the cached keys were last rotated at their plain
+//         window positions. A key enters the cache at window position p during
+//         step k and is rotated once, at angle index p + k*n; every later step
+//         moves it one frame (n positions) towards the start of its view while
+//         k grows by one, so p + k*n stays its angle index for as long as it
+//         is cached. Queries are rotated at their position + k*n. Scores only
+//         depend on angle differences, which equal position differences.
+//   done: blocks of the running insert launch that have finished (reset by the
+//         last one).
+struct RingState {
+    int head;
+    int k;
+    unsigned done;
+    int pad;
+};
+
+__device__ __forceinline__ int2 load_ring_state(const RingState* st) {
+    // L2 (coherence point), never a stale L1 line of an earlier kernel.
+    return __ldcg(reinterpret_cast<const int2*>(st));
+}
 
 // Window position of physical cache row `row` (per kv head).
 // Ring rows: view v, slot s, token i sit at row (v*T + s)*n + i; the slot's
@@ -31,27 +62,28 @@ struct WindowShape {
 // drafted block after them) keep their row index as position: they follow all
 // views. "Keys are stored pre-RoPE and rotated at shifted positions"
 // (FlashDrive technical summary, Methodology 1, "Positional Encoding").
-__host__ __device__ __forceinline__ int key_pos(const WindowShape& w, int row) {
+__host__ __device__ __forceinline__ int key_pos(const WindowShape& w, int head, int row) {
     if (row >= w.ring_rows) return row;
     const int tn = w.T * w.n;
     const int v = row / tn;
     const int rem = row - v * tn;
     const int s = rem / w.n;
     const int i = rem - s * w.n;
-    int age = s - w.head;
+    int age = s - head;
     if (age < 0) age += w.T;
     return v * tn + age * w.n + i;
 }
+__host__ __device__ __forceinline__ int key_pos(const WindowShape& w, int row) { return key_pos(w, w.head, row); }
 
 // Window position of query token t.
 //   prefill: the whole window in order, position t;
 //   step: view v's newest frame (the last of its T frames) then the text,
 //         "inserted at the end of each view's sequence" (FlashDrive technical
 //         summary, Methodology 1, "Token Layout");
-//   verify: a drafted block right after the text.
+//   verify: a drafted block right after the text and the persisted decode tail.
 __host__ __device__ __forceinline__ int query_pos(const WindowShape& w, int mode, int t) {
     if (mode == kQueryPrefill) return t;
-    if (mode == kQueryVerify) return w.ring_rows + w.X + t;
+    if (mode == kQueryVerify) return w.ring_rows + w.X + w.tail + t;
     const int vn = w.V * w.n;
     if (t < vn) {
         const int v = t / w.n;
@@ -70,8 +102,9 @@ struct AttnParams {
     int q_tiles;          // ceil(nq * G / 128)
     int splits;           // key splits per (kv head, query tile)
     float q_scale;        // log2(e) / sqrt(d), folded into the rotated queries
-    const float2* rope;   // [rope_rows][d/2] (cos, sin) of pos * theta_i
+    const float2* rope;   // [rope_rows][d/2] (cos, sin) of angle index * theta_i
     int rope_rows;
+    const RingState* state;  // head and angle offset k (written by kv_stream_insert)
     float* out;           // [nq][H][d] fp32
     float* part_o;        // [items][splits][128][d] fp32 (splits > 1)
     float2* part_ml;      // [items][splits][128] (running max in log2 units, sum)
@@ -79,22 +112,29 @@ struct AttnParams {
     unsigned long long wait_limit_ns;
 };
 
-struct InsertParams {
-    WindowShape w;          // the window after this insert (head advanced): key positions
-    int mode;               // 0: prefill (row = t), 1: step, 2: drafted block (row = L + t)
-    int old_head;           // step: the ring slot each view's new frame overwrites
-    int N;                  // tokens in K_src / V_src
-    int row_begin, row_end; // physical rows processed (whole 128-row tiles, within rows_cap)
-    int key_rows;           // rows [0, key_rows) hold keys; later rows get zero operands
-    int Hkv, d, rows_cap;
+// One layer's buffers for kv_stream_insert.
+struct InsertLayer {
     const uint16_t* K_src;  // [N][Hkv][d] bf16, pre-RoPE
     const uint16_t* V_src;
-    uint16_t* K;            // bf16 cache [Hkv][rows_cap][d]: new rows written, others read
+    uint16_t* K;            // bf16 cache [Hkv][rows_cap][d]: new rows written, others read on a re-base
     uint16_t* V;
-    const float2* rope;     // [rope_rows][d/2] (cos, sin)
     uint16_t* Kh;           // fp16 rotated key, hi part, same layout as the cache
     uint16_t* Kl;           // fp16 rotated key, lo part
     uint16_t* V16;          // fp16 V
+    RingState* state;
+    unsigned* err;          // device error word (kErrRange)
+};
+
+struct InsertParams {
+    WindowShape w;          // window shape (head comes from each layer's state)
+    int mode;               // 0: prefill (row = t), 1: window step, 2: rows [row0, row0 + N) after the text
+    int N;                  // tokens per layer in K_src / V_src
+    int row0;               // mode 2: first physical row written
+    int Hkv, d, rows_cap;
+    int rebase_every;       // R: a window step whose k would reach R re-rotates the whole window (k = 0)
+    const float2* rope;     // [rope_rows][d/2] (cos, sin)
+    int layers;             // entries of `layer` in use (gridDim.y)
+    InsertLayer layer[kMaxInsertBatch];
 };
 
 // Launches `kernel` with programmatic stream serialisation: its launch and set-up
@@ -129,13 +169,16 @@ cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // launch's cudaError_t.
 // kv_stream_insert: new K/V into the bf16 cache, and every processed row's rotated
 // fp16 K hi / lo and fp16 V.
+// One launch covers p.layers layers (blockIdx.y); each block strides over its
+// layer's rows.
 cudaError_t launch_kv_stream_insert(const InsertParams& p, cudaStream_t stream);
 // stream_attn over the rotated operand cache (tkh, tkl, tv16); tq maps the
 // call's bf16 queries [nq][H][d] with box {64, G, 128/G} (128-byte swizzle).
 cudaError_t launch_stream_attn(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkh,
                                const CUtensorMap& tkl, const CUtensorMap& tv16, cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
-cudaError_t launch_positions(const WindowShape& w, int rows, int* pos_out, cudaStream_t stream);
+cudaError_t launch_positions(const WindowShape& w, const RingState* state, int rows, int* pos_out,
+                             cudaStream_t stream);
 cudaError_t launch_wait_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);
 size_t stream_attn_smem_bytes(int d);
 // Fixed split-KV scratch in device memory (no allocation): its capacity in

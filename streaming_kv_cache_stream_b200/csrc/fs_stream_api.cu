@@ -6,11 +6,14 @@
 // in the kernels of kv_stream_insert.cu and stream_attn.cu.
 // Tensor maps are built once per handle (for the cache); queries are read by
 // the kernel with plain loads, so attend encodes nothing per call.
+#include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -27,25 +30,29 @@ struct fs_stream {
     int V, T, n, X, H, Hkv, G, d;
     float base;
     int L, ring_rows, step_tokens, rows_cap, rope_rows;
+    int rebase_every = 16;  // R: every R-th window step re-rotates the whole window
     int state = FS_STATE_EXPECT_PREFILL;
-    int head = 0;
+    int head = 0;           // host mirror of the device ring head (sizes, debug export)
+    int tail = 0;           // persisted decode-tail tokens after the text
     long long steps = 0;
-    int last_insert_tokens = 0;
     std::vector<long long> slot_frame;  // frame id held by each ring slot (same for all views)
     cudaStream_t stream = nullptr;
     int device = 0, num_sms = 148;
-    uint16_t* K_cache = nullptr;  // pre-RoPE bf16 ring + text + drafted-block rows
+    uint16_t* K_cache = nullptr;  // pre-RoPE bf16 ring + text + decode tail + drafted-block rows
     uint16_t* V_cache = nullptr;
-    uint16_t* Kh = nullptr;       // per-step operands: rotated K fp16 hi / lo, V fp16
+    uint16_t* Kh = nullptr;       // attention operands: rotated K fp16 hi / lo, V fp16
     uint16_t* Kl = nullptr;
     uint16_t* V16 = nullptr;
-    float2* rope = nullptr;
+    const float2* rope = nullptr; // shared per (device, d, base, rows); see rope_acquire
+    fs::RingState* dstate = nullptr;  // device-resident ring head and angle offset
     unsigned* err = nullptr;
     float* part_o = nullptr;
     float2* part_ml = nullptr;
     int part_rows_cap = 0;  // rows of 128 query rows x d fp32 the split scratch holds
     void* stage = nullptr;  // host-path staging: K, V, Q, out
     size_t stage_bytes = 0;
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;         // host-path copy streams
+    cudaEvent_t ev_in = nullptr, ev_done = nullptr, ev_out = nullptr;
     CUtensorMap tmap_kh2, tmap_kl2, tmap_v16h;  // fp16 operands, one CTA's half tile (attention loads)
     unsigned long long wait_limit_ns = 2000000000ull;
     long long cache_bytes = 0;
@@ -116,7 +123,62 @@ WindowShape shape_of(const fs_stream* s) {
     w.X = s->X;
     w.ring_rows = s->ring_rows;
     w.head = s->head;
+    w.tail = s->tail;
     return w;
+}
+
+// ---------------------------------------------------------------- RoPE tables
+// cos/sin of (angle index) * base^(-2i/d), evaluated in double, stored as float2
+// [rows][d/2]. Handles of the same device, head dim, base and row count share
+// one table (a 36-layer stack holds one copy, not 36); reference-counted.
+struct RopeEntry {
+    int device, d, rows;
+    float base;
+    float2* ptr;
+    int refs;
+};
+std::mutex g_rope_mu;
+std::vector<RopeEntry> g_rope;
+
+const float2* rope_acquire(int device, int d, float base, int rows, cudaError_t* err) {
+    std::lock_guard<std::mutex> lock(g_rope_mu);
+    for (auto& e : g_rope)
+        if (e.device == device && e.d == d && e.rows == rows && e.base == base) {
+            ++e.refs;
+            return e.ptr;
+        }
+    const size_t bytes = size_t(rows) * (d / 2) * sizeof(float2);
+    std::vector<float2> tab(size_t(rows) * (d / 2));
+    for (int i = 0; i < d / 2; ++i) {
+        const double theta = std::pow(double(base), -2.0 * i / d);
+        for (int a = 0; a < rows; ++a) {
+            const double ang = double(a) * theta;
+            tab[size_t(a) * (d / 2) + i] = make_float2(float(std::cos(ang)), float(std::sin(ang)));
+        }
+    }
+    float2* ptr = nullptr;
+    *err = cudaMalloc(&ptr, bytes);
+    if (*err != cudaSuccess) return nullptr;
+    *err = cudaMemcpy(ptr, tab.data(), bytes, cudaMemcpyHostToDevice);
+    if (*err != cudaSuccess) {
+        cudaFree(ptr);
+        return nullptr;
+    }
+    g_rope.push_back(RopeEntry{device, d, rows, base, ptr, 1});
+    return ptr;
+}
+
+void rope_release(const float2* ptr) {
+    if (!ptr) return;
+    std::lock_guard<std::mutex> lock(g_rope_mu);
+    for (size_t i = 0; i < g_rope.size(); ++i)
+        if (g_rope[i].ptr == ptr) {
+            if (--g_rope[i].refs == 0) {
+                cudaFree(g_rope[i].ptr);
+                g_rope.erase(g_rope.begin() + long(i));
+            }
+            return;
+        }
 }
 
 void free_all(fs_stream* s) {
@@ -125,11 +187,17 @@ void free_all(fs_stream* s) {
     cudaFree(s->Kh);
     cudaFree(s->Kl);
     cudaFree(s->V16);
-    cudaFree(s->rope);
+    rope_release(s->rope);
+    cudaFree(s->dstate);
     cudaFree(s->err);
     cudaFree(s->part_o);
     cudaFree(s->part_ml);
     cudaFree(s->stage);
+    if (s->copy_in) cudaStreamDestroy(s->copy_in);
+    if (s->copy_out) cudaStreamDestroy(s->copy_out);
+    if (s->ev_in) cudaEventDestroy(s->ev_in);
+    if (s->ev_done) cudaEventDestroy(s->ev_done);
+    if (s->ev_out) cudaEventDestroy(s->ev_out);
 }
 
 int check_err_word(fs_stream_t s) {
@@ -138,41 +206,72 @@ int check_err_word(fs_stream_t s) {
     if (h) {
         FS_CUDA(s, cudaMemset(s->err, 0, sizeof(unsigned)));
         if (h & fs::kErrTimeout) return fail(s, FS_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up");
+        if (h & fs::kErrRange)
+            return fail(s, FS_ERR_RANGE,
+                        "an input was out of range: a rotated key, V or scaled rotated query element above 65504 in "
+                        "magnitude, or not finite; outputs since the last check are not valid");
         return fail(s, FS_ERR_CUDA, "device error word 0x%x", h);
     }
     return FS_OK;
 }
 
-// One fused pass (kernel kv_stream_insert): this call's K/V into the cache and
-// every row of the processed range rotated at its position in the window as it
-// stands after the insert (new_head). Prefill and step process every key tile;
-// a drafted block only the tiles from L on (the window's rows were rotated by
-// the last insert and have not moved since).
-int do_insert(fs_stream_t s, const void* K, const void* V, int n_tokens, int mode, int new_head) {
+fs::InsertLayer layer_of(const fs_stream* s, const void* K, const void* V) {
+    fs::InsertLayer ly;
+    ly.K_src = static_cast<const uint16_t*>(K);
+    ly.V_src = static_cast<const uint16_t*>(V);
+    ly.K = s->K_cache;
+    ly.V = s->V_cache;
+    ly.Kh = s->Kh;
+    ly.Kl = s->Kl;
+    ly.V16 = s->V16;
+    ly.state = s->dstate;
+    ly.err = s->err;
+    return ly;
+}
+
+InsertParams insert_params(const fs_stream* s, int mode, int n_tokens, int row0) {
     InsertParams p;
+    std::memset(&p, 0, sizeof p);
     p.w = shape_of(s);
-    p.w.head = new_head;
     p.mode = mode;
-    p.old_head = s->head;
     p.N = n_tokens;
-    p.key_rows = mode == 2 ? s->L + n_tokens : s->L;
-    p.row_begin = mode == 2 ? s->L / fs::kTileRows * fs::kTileRows : 0;
-    p.row_end = (p.key_rows + fs::kTileRows - 1) / fs::kTileRows * fs::kTileRows;
-    if (p.row_end > s->rows_cap) p.row_end = s->rows_cap;
+    p.row0 = row0;
     p.Hkv = s->Hkv;
     p.d = s->d;
     p.rows_cap = s->rows_cap;
-    p.K_src = static_cast<const uint16_t*>(K);
-    p.V_src = static_cast<const uint16_t*>(V);
-    p.K = s->K_cache;
-    p.V = s->V_cache;
+    p.rebase_every = s->rebase_every;
     p.rope = s->rope;
-    p.Kh = s->Kh;
-    p.Kl = s->Kl;
-    p.V16 = s->V16;
+    p.layers = 0;
+    return p;
+}
+
+// One pass of kernel kv_stream_insert for one layer: mode 0 = the whole window
+// (prefill), 1 = a window step (each view's new frame and the text; the device
+// ring state decides whether it is a re-base step that re-rotates the whole
+// window), 2 = n_tokens rows from row0 on (decode tail or drafted block).
+int do_insert(fs_stream_t s, const void* K, const void* V, int n_tokens, int mode, int row0) {
+    InsertParams p = insert_params(s, mode, n_tokens, row0);
+    p.layer[0] = layer_of(s, K, V);
+    p.layers = 1;
     FS_CUDA(s, fs::launch_kv_stream_insert(p, s->stream));
     s->launches += 1;
     return FS_OK;
+}
+
+// Host bookkeeping after a window insert (the device state was advanced by the kernel).
+void after_window_insert(fs_stream_t s, bool prefill) {
+    s->tail = 0;
+    if (prefill) {
+        s->head = 0;
+        s->steps = 0;
+        for (int f = 0; f < s->T; ++f) s->slot_frame[f] = f;
+        s->state = FS_STATE_PREFILLED;
+        return;
+    }
+    s->slot_frame[s->head] = (long long)s->T + s->steps;  // the k-th step inserts frame T-1+k
+    s->head = (s->head + 1) % s->T;
+    s->steps += 1;
+    s->state = FS_STATE_STREAMING;
 }
 
 // Splits of the key range per (kv head, unit of four query tiles) so that
@@ -191,14 +290,9 @@ int choose_splits(const fs_stream* s, int q_tiles, int key_rows) {
     return sp < 1 ? 1 : sp;
 }
 
-int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key_rows) {
-    // Encoded before anything is enqueued, so a failure leaves no partial work.
-    CUtensorMap tq;  // this call's queries, one query tile (128/G tokens x G heads) per box
-    const int rcq = make_map(s, &tq, Q, s->d, s->H, nq, uint64_t(s->d) * 2, uint64_t(s->H) * s->d * 2, s->G,
-                             fs::kTileRows / s->G);
-    if (rcq) return rcq;
-    const int q_tiles = (nq * s->G + fs::kTileRows - 1) / fs::kTileRows;
+AttnParams attn_params(const fs_stream* s, int nq, int mode, int key_rows, void* out) {
     AttnParams p;
+    std::memset(&p, 0, sizeof p);
     p.w = shape_of(s);
     p.key_rows = key_rows;
     p.Hkv = s->Hkv;
@@ -207,22 +301,53 @@ int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key
     p.d = s->d;
     p.nq = nq;
     p.q_mode = mode;
-    p.q_tiles = q_tiles;
-    p.splits = choose_splits(s, q_tiles, key_rows);
+    p.q_tiles = (nq * s->G + fs::kTileRows - 1) / fs::kTileRows;
+    p.splits = 1;
     p.q_scale = float(1.4426950408889634 / std::sqrt(double(s->d)));
     p.rope = s->rope;
     p.rope_rows = s->rope_rows;
+    p.state = s->dstate;
     p.out = static_cast<float*>(out);
     p.part_o = s->part_o;
     p.part_ml = s->part_ml;
     p.err = s->err;
     p.wait_limit_ns = s->wait_limit_ns;
+    return p;
+}
+
+int make_query_map(fs_stream_t s, CUtensorMap* tq, const void* Q, int nq) {
+    // One query tile (128/G tokens x G heads) per box.
+    return make_map(s, tq, Q, s->d, s->H, nq, uint64_t(s->d) * 2, uint64_t(s->H) * s->d * 2, s->G,
+                    fs::kTileRows / s->G);
+}
+
+int launch_attention(fs_stream_t s, const AttnParams& p, const CUtensorMap& tq) {
     FS_CUDA(s, fs::launch_stream_attn(p, tq, s->tmap_kh2, s->tmap_kl2, s->tmap_v16h, s->stream));
     s->launches += 1;
     if (p.splits > 1) {
         FS_CUDA(s, fs::launch_attn_combine(p, s->stream));
         s->launches += 1;
     }
+    return FS_OK;
+}
+
+int do_attend(fs_stream_t s, const void* Q, void* out, int nq, int mode, int key_rows) {
+    // Encoded before anything is enqueued, so a failure leaves no partial work.
+    CUtensorMap tq;
+    const int rcq = make_query_map(s, &tq, Q, nq);
+    if (rcq) return rcq;
+    AttnParams p = attn_params(s, nq, mode, key_rows, out);
+    p.splits = choose_splits(s, p.q_tiles, key_rows);
+    return launch_attention(s, p, tq);
+}
+
+int check_block_args(fs_stream_t s, const void* Q_x, const void* K_x, const void* V_x, int n_x, const void* out) {
+    if (!Q_x || !K_x || !V_x || !out) return fail(s, FS_ERR_ARG, "NULL tensor pointer");
+    if (!aligned16(Q_x) || !aligned16(K_x) || !aligned16(V_x) || !aligned16(out))
+        return fail(s, FS_ERR_ARG, "pointers must be 16-byte aligned");
+    if (n_x < 1 || n_x > FS_MAX_VERIFY_TOKENS) return fail(s, FS_ERR_ARG, "n_x must be in [1, %d]", FS_MAX_VERIFY_TOKENS);
+    if (Q_x == out) return fail(s, FS_ERR_ARG, "out must not alias Q_x");
+    if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "verify before the first insert");
     return FS_OK;
 }
 
@@ -243,8 +368,9 @@ int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame,
     if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return fail(nullptr, FS_ERR_ARG, "rope_base must be > 0");
     const long long ring = (long long)views * frames * tok_per_frame;
     const long long L = ring + text_len;
-    if (L + fs::kMaxVerify > (long long)fs::kMaxKeyTiles * fs::kTileRows)
-        return fail(nullptr, FS_ERR_ARG, "window too long: L + %d must be <= %d", fs::kMaxVerify,
+    const long long extra = fs::kMaxTail + fs::kMaxVerify;
+    if (L + extra > (long long)fs::kMaxKeyTiles * fs::kTileRows)
+        return fail(nullptr, FS_ERR_ARG, "window too long: L + %lld must be <= %d", extra,
                     fs::kMaxKeyTiles * fs::kTileRows);
 
     fs_stream* s = new (std::nothrow) fs_stream();
@@ -261,8 +387,18 @@ int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame,
     s->ring_rows = int(ring);
     s->L = int(L);
     s->step_tokens = views * tok_per_frame + text_len;
-    s->rows_cap = int(L) + fs::kMaxVerify;
-    s->rope_rows = s->rows_cap;
+    s->rows_cap = int(L + extra);
+    if (const char* e = std::getenv("FS_REBASE_STEPS")) {
+        const long v = std::strtol(e, nullptr, 10);
+        if (v >= 1 && v <= 4096) s->rebase_every = int(v);
+    }
+    // Angle indices reach (L + tail + block - 1) + (R - 1) * n.
+    const long long rope_rows = (long long)s->rows_cap + (long long)(s->rebase_every - 1) * tok_per_frame;
+    if (rope_rows > (1ll << 24)) {
+        delete s;
+        return fail(nullptr, FS_ERR_ARG, "RoPE table too large: lower FS_REBASE_STEPS");
+    }
+    s->rope_rows = int(rope_rows);
     s->slot_frame.assign(frames, -1);
     if (const char* e = std::getenv("FS_WAIT_LIMIT_NS")) s->wait_limit_ns = std::strtoull(e, nullptr, 10);
 
@@ -279,33 +415,34 @@ int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame,
     if (major != 10) return bail(fail(nullptr, FS_ERR_CUDA, "needs an sm_100 GPU (B200); found major %d", major));
 
     const size_t cache = size_t(Hkv) * s->rows_cap * d * 2;
-    const size_t rope = size_t(s->rope_rows) * (d / 2) * sizeof(float2);
     s->part_rows_cap = 2 * s->num_sms;
     const size_t part_o = size_t(s->part_rows_cap) * fs::kTileRows * d * sizeof(float);
     const size_t part_ml = size_t(s->part_rows_cap) * fs::kTileRows * sizeof(float2);
     if (cudaMalloc(&s->K_cache, cache) != cudaSuccess || cudaMalloc(&s->V_cache, cache) != cudaSuccess ||
         cudaMalloc(&s->Kh, cache) != cudaSuccess || cudaMalloc(&s->Kl, cache) != cudaSuccess ||
-        cudaMalloc(&s->V16, cache) != cudaSuccess ||
-        cudaMalloc(&s->rope, rope) != cudaSuccess || cudaMalloc(&s->err, sizeof(unsigned)) != cudaSuccess ||
-        cudaMalloc(&s->part_o, part_o) != cudaSuccess || cudaMalloc(&s->part_ml, part_ml) != cudaSuccess) {
+        cudaMalloc(&s->V16, cache) != cudaSuccess || cudaMalloc(&s->dstate, sizeof(fs::RingState)) != cudaSuccess ||
+        cudaMalloc(&s->err, sizeof(unsigned)) != cudaSuccess || cudaMalloc(&s->part_o, part_o) != cudaSuccess ||
+        cudaMalloc(&s->part_ml, part_ml) != cudaSuccess) {
         cudaGetLastError();
-        return bail(fail(nullptr, FS_ERR_OOM, "device allocation of %zu bytes failed", 5 * cache + rope + part_o));
+        return bail(fail(nullptr, FS_ERR_OOM, "device allocation of %zu bytes failed", 5 * cache + part_o));
     }
-    s->cache_bytes = (long long)(5 * cache + rope + part_o + part_ml + sizeof(unsigned));
+    // Every operand row starts finite (zero): rows past a call's last key are
+    // masked by position, and 0 x finite stays 0 in P V.
     if (cudaMemset(s->K_cache, 0, cache) != cudaSuccess || cudaMemset(s->V_cache, 0, cache) != cudaSuccess ||
+        cudaMemset(s->Kh, 0, cache) != cudaSuccess || cudaMemset(s->Kl, 0, cache) != cudaSuccess ||
+        cudaMemset(s->V16, 0, cache) != cudaSuccess || cudaMemset(s->dstate, 0, sizeof(fs::RingState)) != cudaSuccess ||
         cudaMemset(s->err, 0, sizeof(unsigned)) != cudaSuccess)
         return bail(fail(nullptr, FS_ERR_CUDA, "cudaMemset failed"));
-
-    // RoPE table: cos/sin of pos * base^(-2i/d), evaluated in double, stored as float.
-    std::vector<float2> tab(size_t(s->rope_rows) * (d / 2));
-    for (int pos = 0; pos < s->rope_rows; ++pos)
-        for (int i = 0; i < d / 2; ++i) {
-            const double theta = std::pow(double(rope_base), -2.0 * i / d);
-            const double a = double(pos) * theta;
-            tab[size_t(pos) * (d / 2) + i] = make_float2(float(std::cos(a)), float(std::sin(a)));
-        }
-    if (cudaMemcpy(s->rope, tab.data(), rope, cudaMemcpyHostToDevice) != cudaSuccess)
-        return bail(fail(nullptr, FS_ERR_CUDA, "RoPE table upload failed"));
+    e = cudaSuccess;
+    s->rope = rope_acquire(s->device, d, rope_base, s->rope_rows, &e);
+    if (!s->rope) {
+        cudaGetLastError();
+        return bail(fail(nullptr, e == cudaErrorMemoryAllocation ? FS_ERR_OOM : FS_ERR_CUDA,
+                         "RoPE table (%d rows) failed: %s", s->rope_rows, cudaGetErrorString(e)));
+    }
+    const size_t rope = size_t(s->rope_rows) * (d / 2) * sizeof(float2);
+    s->cache_bytes = (long long)(5 * cache + part_o + part_ml + sizeof(unsigned) + sizeof(fs::RingState));
+    (void)rope;
 
     const uint64_t row_bytes = uint64_t(d) * 2;
     const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -326,6 +463,8 @@ int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame,
 int fs_stream_destroy(fs_stream_t s) {
     if (!s) return FS_OK;
     cudaStreamSynchronize(s->stream);
+    if (s->copy_in) cudaStreamSynchronize(s->copy_in);
+    if (s->copy_out) cudaStreamSynchronize(s->copy_out);
     free_all(s);
     delete s;
     return FS_OK;
@@ -341,6 +480,7 @@ int fs_stream_reset(fs_stream_t s) {
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
     s->state = FS_STATE_EXPECT_PREFILL;
     s->head = 0;
+    s->tail = 0;
     s->steps = 0;
     s->slot_frame.assign(s->T, -1);
     return FS_OK;
@@ -350,22 +490,43 @@ int fs_stream_insert(fs_stream_t s, const void* K_new, const void* V_new) {
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
     if (!K_new || !V_new) return fail(s, FS_ERR_ARG, "K_new/V_new is NULL");
     if (!aligned16(K_new) || !aligned16(V_new)) return fail(s, FS_ERR_ARG, "K_new/V_new must be 16-byte aligned");
-    if (s->state == FS_STATE_EXPECT_PREFILL) {
-        s->head = 0;
-        int rc = do_insert(s, K_new, V_new, s->L, 0, 0);
-        if (rc) return rc;
-        for (int f = 0; f < s->T; ++f) s->slot_frame[f] = f;
-        s->state = FS_STATE_PREFILLED;
-        s->last_insert_tokens = s->L;
-        return FS_OK;
-    }
-    int rc = do_insert(s, K_new, V_new, s->step_tokens, 1, (s->head + 1) % s->T);
+    const bool prefill = s->state == FS_STATE_EXPECT_PREFILL;
+    int rc = do_insert(s, K_new, V_new, prefill ? s->L : s->step_tokens, prefill ? 0 : 1, 0);
     if (rc) return rc;
-    s->slot_frame[s->head] = (long long)s->T + s->steps;  // the k-th step inserts frame T-1+k
-    s->head = (s->head + 1) % s->T;
-    s->steps += 1;
-    s->state = FS_STATE_STREAMING;
-    s->last_insert_tokens = s->step_tokens;
+    after_window_insert(s, prefill);
+    return FS_OK;
+}
+
+int fs_stream_insert_batch(fs_stream_t* handles, int n, const void* const* K_new, const void* const* V_new) {
+    if (!handles || !K_new || !V_new || n < 1) return fail(nullptr, FS_ERR_ARG, "NULL array or n < 1");
+    fs_stream_t s0 = handles[0];
+    if (!s0) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    const bool prefill = s0->state == FS_STATE_EXPECT_PREFILL;
+    for (int i = 0; i < n; ++i) {
+        fs_stream_t s = handles[i];
+        if (!s) return fail(s0, FS_ERR_ARG, "handle %d is NULL", i);
+        if (!K_new[i] || !V_new[i] || !aligned16(K_new[i]) || !aligned16(V_new[i]))
+            return fail(s0, FS_ERR_ARG, "K_new/V_new of layer %d NULL or not 16-byte aligned", i);
+        if (s->V != s0->V || s->T != s0->T || s->n != s0->n || s->X != s0->X || s->Hkv != s0->Hkv ||
+            s->d != s0->d || s->rows_cap != s0->rows_cap || s->rebase_every != s0->rebase_every ||
+            s->rope != s0->rope || s->device != s0->device)
+            return fail(s0, FS_ERR_ARG, "handle %d differs in shape, RoPE table or device from handle 0", i);
+        if (s->stream != s0->stream) return fail(s0, FS_ERR_ARG, "handle %d is on another stream", i);
+        if ((s->state == FS_STATE_EXPECT_PREFILL) != prefill)
+            return fail(s0, FS_ERR_STATE, "handles mix prefill and window-step states (handle %d)", i);
+        for (int j = 0; j < i; ++j)
+            if (handles[j] == s) return fail(s0, FS_ERR_ARG, "handle %d appears twice", i);
+    }
+    const int tokens = prefill ? s0->L : s0->step_tokens;
+    for (int b = 0; b < n; b += fs::kMaxInsertBatch) {
+        const int cnt = n - b < fs::kMaxInsertBatch ? n - b : fs::kMaxInsertBatch;
+        InsertParams p = insert_params(s0, prefill ? 0 : 1, tokens, 0);
+        for (int i = 0; i < cnt; ++i) p.layer[i] = layer_of(handles[b + i], K_new[b + i], V_new[b + i]);
+        p.layers = cnt;
+        FS_CUDA(s0, fs::launch_kv_stream_insert(p, s0->stream));
+        s0->launches += 1;
+    }
+    for (int i = 0; i < n; ++i) after_window_insert(handles[i], prefill);
     return FS_OK;
 }
 
@@ -379,17 +540,34 @@ int fs_stream_attend(fs_stream_t s, const void* Q, void* out) {
     return do_attend(s, Q, out, pre ? s->L : s->step_tokens, pre ? fs::kQueryPrefill : fs::kQueryStep, s->L);
 }
 
+int fs_stream_append(fs_stream_t s, const void* K_acc, const void* V_acc, int n_acc) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (!K_acc || !V_acc) return fail(s, FS_ERR_ARG, "K_acc/V_acc is NULL");
+    if (!aligned16(K_acc) || !aligned16(V_acc)) return fail(s, FS_ERR_ARG, "K_acc/V_acc must be 16-byte aligned");
+    if (n_acc < 1) return fail(s, FS_ERR_ARG, "n_acc must be >= 1");
+    if (s->tail + n_acc > FS_MAX_TAIL_TOKENS)
+        return fail(s, FS_ERR_ARG, "decode tail would hold %d tokens; the limit is %d", s->tail + n_acc,
+                    FS_MAX_TAIL_TOKENS);
+    if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "append before the first insert");
+    int rc = do_insert(s, K_acc, V_acc, n_acc, 2, s->L + s->tail);
+    if (rc) return rc;
+    s->tail += n_acc;
+    return FS_OK;
+}
+
 int fs_stream_attend_ext(fs_stream_t s, const void* Q_x, const void* K_x, const void* V_x, int n_x, void* out) {
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
-    if (!Q_x || !K_x || !V_x || !out) return fail(s, FS_ERR_ARG, "NULL tensor pointer");
-    if (!aligned16(Q_x) || !aligned16(K_x) || !aligned16(V_x) || !aligned16(out))
-        return fail(s, FS_ERR_ARG, "pointers must be 16-byte aligned");
-    if (n_x < 1 || n_x > FS_MAX_VERIFY_TOKENS) return fail(s, FS_ERR_ARG, "n_x must be in [1, %d]", FS_MAX_VERIFY_TOKENS);
-    if (Q_x == out) return fail(s, FS_ERR_ARG, "out must not alias Q_x");
-    if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "verify before the first insert");
-    int rc = do_insert(s, K_x, V_x, n_x, 2, s->head);
+    int rc = check_block_args(s, Q_x, K_x, V_x, n_x, out);
     if (rc) return rc;
-    return do_attend(s, Q_x, out, n_x, fs::kQueryVerify, s->L + n_x);
+    CUtensorMap tq;
+    rc = make_query_map(s, &tq, Q_x, n_x);
+    if (rc) return rc;
+    const int key_rows = s->L + s->tail + n_x;
+    rc = do_insert(s, K_x, V_x, n_x, 2, s->L + s->tail);
+    if (rc) return rc;
+    AttnParams p = attn_params(s, n_x, fs::kQueryVerify, key_rows, out);
+    p.splits = choose_splits(s, p.q_tiles, key_rows);
+    return launch_attention(s, p, tq);
 }
 
 // Same computation as fs_stream_attend_ext, with the split-KV partials in the
@@ -404,15 +582,12 @@ int fs_stream_attend_ext(fs_stream_t s, const void* Q_x, const void* K_x, const 
 int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x, const void* V_x, int n_x,
                                 void* out) {
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
-    if (!Q_x || !K_x || !V_x || !out) return fail(s, FS_ERR_ARG, "NULL tensor pointer");
-    if (!aligned16(Q_x) || !aligned16(K_x) || !aligned16(V_x) || !aligned16(out))
-        return fail(s, FS_ERR_ARG, "pointers must be 16-byte aligned");
-    if (n_x < 1 || n_x > FS_MAX_VERIFY_TOKENS) return fail(s, FS_ERR_ARG, "n_x must be in [1, %d]", FS_MAX_VERIFY_TOKENS);
-    if (Q_x == out) return fail(s, FS_ERR_ARG, "out must not alias Q_x");
-    if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "verify before the first insert");
-    const int key_rows = s->L + n_x;
+    int rc = check_block_args(s, Q_x, K_x, V_x, n_x, out);
+    if (rc) return rc;
+    const int key_rows = s->L + s->tail + n_x;
     const int q_tiles = (n_x * s->G + fs::kTileRows - 1) / fs::kTileRows;
-    // Partial tiles per split, counted as choose_splits does (query tiles padded to pairs).
+    // Partial tiles per split, a deliberate upper bound: query tiles padded to
+    // whole pairs (the kernel writes q_tiles * Hkv of them).
     const int tiles_padded = 2 * ((q_tiles + 1) / 2) * s->Hkv;
     const int cap = fs::static_split_scratch_tiles();
     if (tiles_padded > cap)
@@ -425,40 +600,26 @@ int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x,
     float* part_o = nullptr;
     float2* part_ml = nullptr;
     FS_CUDA(s, fs::static_split_scratch(&part_o, &part_ml));
-    CUtensorMap tq;  // this call's queries, one query tile (128/G tokens x G heads) per box
-    const int rcq = make_map(s, &tq, Q_x, s->d, s->H, n_x, uint64_t(s->d) * 2, uint64_t(s->H) * s->d * 2, s->G,
-                             fs::kTileRows / s->G);
-    if (rcq) return rcq;
-    int rc = do_insert(s, K_x, V_x, n_x, 2, s->head);
+    CUtensorMap tq;
+    rc = make_query_map(s, &tq, Q_x, n_x);
     if (rc) return rc;
-    AttnParams p;
-    p.w = shape_of(s);
-    p.key_rows = key_rows;
-    p.Hkv = s->Hkv;
-    p.G = s->G;
-    p.H = s->H;
-    p.d = s->d;
-    p.nq = n_x;
-    p.q_mode = fs::kQueryVerify;
-    p.q_tiles = q_tiles;
+    rc = do_insert(s, K_x, V_x, n_x, 2, s->L + s->tail);
+    if (rc) return rc;
+    AttnParams p = attn_params(s, n_x, fs::kQueryVerify, key_rows, out);
     p.splits = splits;
-    p.q_scale = float(1.4426950408889634 / std::sqrt(double(s->d)));
-    p.rope = s->rope;
-    p.rope_rows = s->rope_rows;
-    p.out = static_cast<float*>(out);
     p.part_o = part_o;
     p.part_ml = part_ml;
-    p.err = s->err;
-    p.wait_limit_ns = s->wait_limit_ns;
-    FS_CUDA(s, fs::launch_stream_attn(p, tq, s->tmap_kh2, s->tmap_kl2, s->tmap_v16h, s->stream));
-    s->launches += 1;
-    if (p.splits > 1) {
-        FS_CUDA(s, fs::launch_attn_combine(p, s->stream));
-        s->launches += 1;
-    }
-    return FS_OK;
+    return launch_attention(s, p, tq);
 }
 
+// Insert + attend from host buffers. Three streams keep the copy engines and
+// the SMs busy at once: the handle's own copy-in stream stages this call's
+// K/V/Q (after the previous call's kernels have consumed the staging buffer),
+// the caller's stream runs the kernels once those copies have landed (and the
+// previous call's output has left the staging buffer), and the handle's
+// copy-out stream returns the output. Consecutive calls on different handles
+// (layers) therefore overlap one layer's upload, another's kernels and a
+// third's download; fs_stream_sync waits for all three streams.
 int fs_stream_step_host(fs_stream_t s, const void* K_new_h, const void* V_new_h, const void* Q_h, void* out_h) {
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
     if (!K_new_h || !V_new_h || !Q_h || !out_h) return fail(s, FS_ERR_ARG, "NULL host pointer");
@@ -467,9 +628,18 @@ int fs_stream_step_host(fs_stream_t s, const void* K_new_h, const void* V_new_h,
     const size_t qb = size_t(nt) * s->H * s->d * 2;  // Q, bf16
     const size_t ob = 2 * qb;                           // out, fp32
     const size_t need = 2 * kv + qb + ob + 4 * 256;
+    if (!s->copy_in) {
+        FS_CUDA(s, cudaStreamCreateWithFlags(&s->copy_in, cudaStreamNonBlocking));
+        FS_CUDA(s, cudaStreamCreateWithFlags(&s->copy_out, cudaStreamNonBlocking));
+        FS_CUDA(s, cudaEventCreateWithFlags(&s->ev_in, cudaEventDisableTiming));
+        FS_CUDA(s, cudaEventCreateWithFlags(&s->ev_done, cudaEventDisableTiming));
+        FS_CUDA(s, cudaEventCreateWithFlags(&s->ev_out, cudaEventDisableTiming));
+    }
     if (need > s->stage_bytes) {
         // Grown on first use (sized for the largest call so far), outside any capture.
         FS_CUDA(s, cudaStreamSynchronize(s->stream));
+        FS_CUDA(s, cudaStreamSynchronize(s->copy_in));
+        FS_CUDA(s, cudaStreamSynchronize(s->copy_out));
         cudaFree(s->stage);
         s->stage = nullptr;
         s->stage_bytes = 0;
@@ -485,20 +655,32 @@ int fs_stream_step_host(fs_stream_t s, const void* K_new_h, const void* V_new_h,
     void* dV = base + up(kv);
     void* dQ = base + 2 * up(kv);
     void* dO = base + 2 * up(kv) + up(qb);
-    FS_CUDA(s, cudaMemcpyAsync(dK, K_new_h, kv, cudaMemcpyHostToDevice, s->stream));
-    FS_CUDA(s, cudaMemcpyAsync(dV, V_new_h, kv, cudaMemcpyHostToDevice, s->stream));
-    FS_CUDA(s, cudaMemcpyAsync(dQ, Q_h, qb, cudaMemcpyHostToDevice, s->stream));
+    // Inputs: after the previous call's kernels have read the staging buffer.
+    FS_CUDA(s, cudaStreamWaitEvent(s->copy_in, s->ev_done, 0));
+    FS_CUDA(s, cudaMemcpyAsync(dK, K_new_h, kv, cudaMemcpyHostToDevice, s->copy_in));
+    FS_CUDA(s, cudaMemcpyAsync(dV, V_new_h, kv, cudaMemcpyHostToDevice, s->copy_in));
+    FS_CUDA(s, cudaMemcpyAsync(dQ, Q_h, qb, cudaMemcpyHostToDevice, s->copy_in));
+    FS_CUDA(s, cudaEventRecord(s->ev_in, s->copy_in));
+    // Kernels: after the inputs landed and the previous output left.
+    FS_CUDA(s, cudaStreamWaitEvent(s->stream, s->ev_in, 0));
+    FS_CUDA(s, cudaStreamWaitEvent(s->stream, s->ev_out, 0));
     int rc = fs_stream_insert(s, dK, dV);
     if (rc) return rc;
     rc = fs_stream_attend(s, dQ, dO);
     if (rc) return rc;
-    FS_CUDA(s, cudaMemcpyAsync(out_h, dO, ob, cudaMemcpyDeviceToHost, s->stream));
+    FS_CUDA(s, cudaEventRecord(s->ev_done, s->stream));
+    // Output.
+    FS_CUDA(s, cudaStreamWaitEvent(s->copy_out, s->ev_done, 0));
+    FS_CUDA(s, cudaMemcpyAsync(out_h, dO, ob, cudaMemcpyDeviceToHost, s->copy_out));
+    FS_CUDA(s, cudaEventRecord(s->ev_out, s->copy_out));
     return FS_OK;
 }
 
 int fs_stream_sync(fs_stream_t s) {
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
     FS_CUDA(s, cudaStreamSynchronize(s->stream));
+    if (s->copy_in) FS_CUDA(s, cudaStreamSynchronize(s->copy_in));
+    if (s->copy_out) FS_CUDA(s, cudaStreamSynchronize(s->copy_out));
     return check_err_word(s);
 }
 
@@ -520,6 +702,8 @@ int fs_stream_info(fs_stream_t s, fs_stream_info_t* info) {
     info->steps = s->steps;
     info->cache_bytes = s->cache_bytes;
     info->launches = s->launches;
+    info->tail_tokens = s->tail;
+    info->rebase_every = s->rebase_every;
     return FS_OK;
 }
 
@@ -527,7 +711,7 @@ int fs_stream_debug_export(fs_stream_t s, void* K_phys, void* V_phys, int32_t* p
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
     if (s->state == FS_STATE_EXPECT_PREFILL) return fail(s, FS_ERR_STATE, "nothing inserted yet");
     FS_CUDA(s, cudaStreamSynchronize(s->stream));
-    const int rows = s->L;
+    const int rows = s->L + s->tail;
     const size_t row_bytes = size_t(s->d) * 2;
     for (int h = 0; h < s->Hkv; ++h) {
         const size_t src = size_t(h) * s->rows_cap * row_bytes;
@@ -540,10 +724,11 @@ int fs_stream_debug_export(fs_stream_t s, void* K_phys, void* V_phys, int32_t* p
                                   rows * row_bytes, cudaMemcpyDeviceToHost));
     }
     if (pos_phys) {
-        // Positions as the attention kernel derives them (same device function).
+        // Positions as the attention kernel derives them (same device function,
+        // head from the device-resident ring state).
         int* dpos = nullptr;
         FS_CUDA(s, cudaMalloc(&dpos, size_t(rows) * sizeof(int)));
-        cudaError_t e = fs::launch_positions(shape_of(s), rows, dpos, s->stream);
+        cudaError_t e = fs::launch_positions(shape_of(s), s->dstate, rows, dpos, s->stream);
         if (e == cudaSuccess) e = cudaStreamSynchronize(s->stream);
         if (e == cudaSuccess) e = cudaMemcpy(pos_phys, dpos, size_t(rows) * sizeof(int), cudaMemcpyDeviceToHost);
         cudaFree(dpos);

@@ -14,9 +14,10 @@
 // the V columns) and multiplied against both groups, so the pair reads 96 KB
 // of operands per 512 query rows: on B200 the tensor pipes of all SMs would
 // otherwise need more from L2 than it delivers. A query tile packs 128/G
-// tokens x the G query heads of one kv group (GQA). The keys were rotated for
-// this step by kv_stream_insert (at their shifted positions, as fp16 hi + lo;
-// V as fp16); this kernel rotates its query rows.
+// tokens x the G query heads of one kv group (GQA). The keys were rotated once
+// by kv_stream_insert (fp16 hi + lo at angle index position + k*n, k the ring
+// state's step count; V as fp16); this kernel rotates its query rows at their
+// positions + k*n, read from the device-resident ring state.
 //
 // Warp roles per CTA (12 warps):
 //   warps 0-3   prologue: classify the key tiles against the unit's and each
@@ -96,7 +97,7 @@ constexpr int kMaskWords = kMaxKeyTiles / 32;
 struct Ctrl {
     uint64_t bars[kNumBars];
     alignas(16) int kpos[kTileRows];     // key positions of the tile being masked
-    uint16_t red_m[2][2][kTileRows];     // [group][column half][row]: partial row max (bf16, rounded up)
+    uint16_t red_m[2][2][kTileRows];     // [group][column half][row]: partial row max, 16 bits at a time
     uint32_t vis[kMaskWords];            // key tile visible to some query of the pair
     uint32_t part[2][kMaskWords];        // per group: tile needs the elementwise mask
     uint32_t tmem_base;
@@ -132,7 +133,7 @@ struct Layout {
 // Lowest and highest window position among physical key rows [r0, r1). Rows of
 // one ring slot (or the text) are consecutive positions, so walking slot-sized
 // runs is exact.
-__device__ __forceinline__ void key_bounds(const WindowShape& w, int r0, int r1, int& lo, int& hi) {
+__device__ __forceinline__ void key_bounds(const WindowShape& w, int head, int r0, int r1, int& lo, int& hi) {
     lo = INT_MAX;
     hi = INT_MIN;
     int r = r0;
@@ -142,7 +143,7 @@ __device__ __forceinline__ void key_bounds(const WindowShape& w, int r0, int r1,
             const int slot_end = (r / w.n + 1) * w.n;
             end = slot_end < r1 ? slot_end : r1;
         }
-        const int a = key_pos(w, r);
+        const int a = key_pos(w, head, r);
         const int b = a + (end - 1 - r);
         lo = a < lo ? a : lo;
         hi = b > hi ? b : hi;
@@ -163,7 +164,7 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 // Pair (i, i + D/2): for D = 128 chunk c of region 0 pairs with chunk c of
 // region 1; for D = 64 chunk c pairs with chunk c + 4.
 template <int D, typename Ready>
-__device__ __forceinline__ void rope_query_row(const float2* __restrict__ cs, float scale, uint8_t* qhi, uint8_t* qlo,
+__device__ __forceinline__ bool rope_query_row(const float2* __restrict__ cs, float scale, uint8_t* qhi, uint8_t* qlo,
                                                int row, Ready ready) {
     constexpr int kPairs = D / 16;  // 16-byte chunk pairs (c, c + D/16) of the row
     constexpr int kHalf = kPairs / 2;
@@ -177,6 +178,7 @@ __device__ __forceinline__ void rope_query_row(const float2* __restrict__ cs, fl
     const bool ok = ready();  // on a timeout the rows rotate whatever is there; the error is reported
     (void)ok;
     // Read the whole bf16 row before overwriting its lo half in place.
+    bool in_range = true;  // every element finite and at most 65504 in magnitude (NaN fails too)
     uint4 a[kPairs], b[kPairs];
 #pragma unroll
     for (int c = 0; c < kPairs; ++c) {
@@ -204,14 +206,19 @@ __device__ __forceinline__ void rope_query_row(const float2* __restrict__ cs, fl
             const float4 tq = t[u][q];  // (cos, sin) of elements 8c + 2q and 8c + 2q + 1
             const float x0 = bf16lo(aw[q]), x1 = bf16hi(aw[q]);
             const float y0 = bf16lo(bw[q]), y1 = bf16hi(bw[q]);
-            split2((x0 * tq.x - y0 * tq.y) * scale, (x1 * tq.z - y1 * tq.w) * scale, ah[q], al[q]);
-            split2((y0 * tq.x + x0 * tq.y) * scale, (y1 * tq.z + x1 * tq.w) * scale, bh[q], bl[q]);
+            const float r0 = (x0 * tq.x - y0 * tq.y) * scale, r1 = (x1 * tq.z - y1 * tq.w) * scale;
+            const float s0 = (y0 * tq.x + x0 * tq.y) * scale, s1 = (y1 * tq.z + x1 * tq.w) * scale;
+            in_range = in_range && fabsf(r0) <= kF16Max && fabsf(r1) <= kF16Max && fabsf(s0) <= kF16Max &&
+                       fabsf(s1) <= kF16Max;
+            split2(r0, r1, ah[q], al[q]);
+            split2(s0, s1, bh[q], bl[q]);
         }
         *reinterpret_cast<uint4*>(qhi + oa) = make_uint4(ah[0], ah[1], ah[2], ah[3]);
         *reinterpret_cast<uint4*>(qhi + ob) = make_uint4(bh[0], bh[1], bh[2], bh[3]);
         *reinterpret_cast<uint4*>(qlo + oa) = make_uint4(al[0], al[1], al[2], al[3]);
         *reinterpret_cast<uint4*>(qlo + ob) = make_uint4(bl[0], bl[1], bl[2], bl[3]);
     }
+    return in_range;
 }
 
 // Uniform decision over `threads` threads at named barrier `id`: true iff all pass `ok`.
@@ -275,6 +282,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     grid_dependency_wait();     // the insert that wrote this call's operands is done
     allow_dependents_launch();  // the next kernel may start its set-up
+    // Ring head and angle offset as the last insert left them (the window shape
+    // itself stays in the parameter space).
+    const WindowShape& w = p.w;
+    int head, angle_off;
+    {
+        const int2 rs = load_ring_state(p.state);
+        head = rs.x;
+        angle_off = rs.y * w.n;
+    }
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -292,7 +308,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int tpt = kTileRows / p.G;  // tokens per query tile
     const int unit_t0 = 4 * u * tpt;
     const int unit_t1 = min(unit_t0 + 4 * tpt, p.nq);
-    const int unit_qmax = query_pos(p.w, p.q_mode, unit_t1 - 1);
+    const int unit_qmax = query_pos(w, p.q_mode, unit_t1 - 1);
     const BoundedWait wait{p.err, p.wait_limit_ns, kErrTimeout};
 
     auto bar = [&](int i) { return smem_u32(&ctrl.bars[i]); };
@@ -367,8 +383,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int t0 = unit_t0 + 2 * g * tpt;
                 const int t1 = min(t0 + 2 * tpt, p.nq);
                 gpresent[g] = t0 < t1;
-                gmin[g] = gpresent[g] ? query_pos(p.w, p.q_mode, t0) : 0;
-                gmax[g] = gpresent[g] ? query_pos(p.w, p.q_mode, t1 - 1) : 0;
+                gmin[g] = gpresent[g] ? query_pos(w, p.q_mode, t0) : 0;
+                gmax[g] = gpresent[g] ? query_pos(w, p.q_mode, t1 - 1) : 0;
             }
             const int words = (n_ktiles + 31) >> 5;
             for (int wd = warp; wd < words; wd += 4) {
@@ -378,7 +394,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const int r0 = j * kTileRows;
                     const int r1 = min(r0 + kTileRows, p.key_rows);
                     int lo, hi;
-                    key_bounds(p.w, r0, r1, lo, hi);
+                    key_bounds(w, head, r0, r1, lo, hi);
                     v = lo <= unit_qmax;
                     const bool full_tile = r1 - r0 == kTileRows;
                     pa = !(gpresent[0] && hi <= gmin[0] && full_tile);
@@ -533,10 +549,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // Rotate this group's query rows (landed by TMA) in shared memory while
             // warps 0-3 classify the key tiles; rows past the last token rotate
             // zeros and are never stored.
-            const int qp0 = query_pos(p.w, p.q_mode, (tile_valid && t < p.nq) ? t : unit_t0);
+            const int qp0 = query_pos(w, p.q_mode, (tile_valid && t < p.nq) ? t : unit_t0);
             uint8_t* qg = smem + L::kQ + 2 * grp * L::kQHalf;
-            rope_query_row<D>(p.rope + (size_t)qp0 * (D / 2), p.q_scale, qg, qg + L::kQHalf, r,
-                              [&] { return wait(bar(kBarQLoad), 0); });
+            const bool in_range =
+                rope_query_row<D>(p.rope + (size_t)(qp0 + angle_off) * (D / 2), p.q_scale, qg, qg + L::kQHalf, r,
+                                  [&] { return wait(bar(kBarQLoad), 0); });
+            if (!in_range && tile_valid && t < p.nq) atomicOr(p.err, kErrRange);
             fence_proxy_async_smem();  // generic stores -> read by the tensor core
         }
         prologue_sync(false);
@@ -545,9 +563,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ---- softmax: both warpgroups on every S tile of both groups; warpgroup
         // hw takes columns [64 hw, 64 hw + 64) of the 128 keys (two warps per SM
         // sub-partition on each tile). The halves agree on the row max through
-        // shared memory (each half's max rounded up to bf16, so both compute the
-        // same value; any base at or above the true max keeps P <= 1), keep their
-        // own partial row sums, and rescale their own D/2 columns of O.
+        // shared memory (see the exchange below: both compute the same base, at
+        // or above the true max, so P <= 1), keep their own partial row sums,
+        // and rescale their own D/2 columns of O.
         const int hw = grp;                // column half (the warpgroup)
         int qpos[2];                       // this row's query position in group g (-1: no query)
         bool rvalid[2];
@@ -556,7 +574,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int qtg = 4 * u + 2 * g + int(rank);
             const int tg = qtg * tpt + r / p.G;
             rvalid[g] = qtg < p.q_tiles && tg < p.nq;
-            qpos[g] = rvalid[g] ? query_pos(p.w, p.q_mode, tg) : -1;
+            qpos[g] = rvalid[g] ? query_pos(w, p.q_mode, tg) : -1;
         }
         float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
         bool ok = true;
@@ -569,7 +587,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // streaming mask (the same key tile serves both groups).
                 if (hw == 0) {
                     const int row = j * kTileRows + r;
-                    ctrl.kpos[r] = row < p.key_rows ? key_pos(p.w, row) : INT_MAX;
+                    ctrl.kpos[r] = row < p.key_rows ? key_pos(w, head, row) : INT_MAX;
                 }
                 named_bar_sync(5, 256);
             }
@@ -604,6 +622,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     mx[(c >> 1) & 7] = fmax3(mx[(c >> 1) & 7], __uint_as_float(sr[c >> 5][c & 31]),
                                              __uint_as_float(sr[c >> 5][(c + 1) & 31]));
                 const float mh = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+                // Row max over both halves, exchanged through shared memory: each
+                // half stores its maximum rounded up to bf16 and both take the
+                // larger, so they agree on one base at or above the true row max
+                // (P <= 1). Rounding up by at most 2^-8 of the value keeps the base
+                // within 1 of the true max while |max| < 256 (log2 units); beyond
+                // that the base could overshoot enough to flush every P to zero,
+                // so such rows exchange their exact fp32 maxima, 16 bits at a time.
                 ctrl.red_m[g][hw][r] = bf16_round_up(mh);
                 // Exchange point, and the uniform decision: a failed wait anywhere
                 // ends the loop for all 256 threads together.
@@ -611,7 +636,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                const float mt = fmaxf(bf16_to_float(ctrl.red_m[g][0][r]), bf16_to_float(ctrl.red_m[g][1][r]));
+                float mt = fmaxf(bf16_to_float(ctrl.red_m[g][0][r]), bf16_to_float(ctrl.red_m[g][1][r]));
+                // The two halves of these 32 rows are warps (warp & 3) and (warp & 3) + 4
+                // of the two warpgroups; both see the same stored values, so they
+                // take this branch together and meet at their own named barrier.
+                if (__any_sync(0xffffffffu, !(fabsf(mt) < 256.f) && mt != -INFINITY)) {
+                    const uint32_t pair_bar = 7u + uint32_t(warp & 3);
+                    const uint32_t bits = __float_as_uint(mh);
+                    named_bar_sync(pair_bar, 64);  // both halves have read the rounded values
+                    ctrl.red_m[g][hw][r] = uint16_t(bits >> 16);
+                    named_bar_sync(pair_bar, 64);
+                    const uint32_t hi = ctrl.red_m[g][hw ^ 1][r];
+                    named_bar_sync(pair_bar, 64);
+                    ctrl.red_m[g][hw][r] = uint16_t(bits & 0xFFFFu);
+                    named_bar_sync(pair_bar, 64);
+                    const uint32_t lo = ctrl.red_m[g][hw ^ 1][r];
+                    mt = fmaxf(mh, __uint_as_float((hi << 16) | lo));  // same value in both halves
+                }
                 const float m_new = fmaxf(m_run[g], mt);
                 const bool resc = m_new > m_run[g] + kRescaleLog2;
                 const float m_use = resc ? m_new : m_run[g];
@@ -773,7 +814,11 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
     for (int e = 0; e < kPer; ++e) dst[e] = acc[e] * inv;
 }
 
-__global__ void positions_kernel(const WindowShape w, int rows, int* pos) {
+// Window positions of physical rows [0, rows) as the attention kernel derives
+// them (same function, head read from the device-resident ring state).
+__global__ void positions_kernel(const WindowShape w0, const RingState* state, int rows, int* pos) {
+    WindowShape w = w0;
+    w.head = load_ring_state(state).x;
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < rows) pos[i] = key_pos(w, i);
 }
@@ -826,9 +871,10 @@ cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_positions(const WindowShape& w, int rows, int* pos_out, cudaStream_t stream) {
+cudaError_t launch_positions(const WindowShape& w, const RingState* state, int rows, int* pos_out,
+                             cudaStream_t stream) {
     if (rows <= 0) return cudaSuccess;
-    positions_kernel<<<(rows + 255) / 256, 256, 0, stream>>>(w, rows, pos_out);
+    positions_kernel<<<(rows + 255) / 256, 256, 0, stream>>>(w, state, rows, pos_out);
     return cudaGetLastError();
 }
 

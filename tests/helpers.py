@@ -62,14 +62,18 @@ def check_cache_bitexact(stream, orc: StreamOracle, wl) -> None:
     for row, (v, f, t) in enumerate(zip(c["view"], c["frame_id"], c["token"])):
         idx[(int(v), int(f), int(t))] = row
     rows = ex["pos"].shape[0]
+    assert rows == c["K"].shape[0], f"device holds {rows} rows, oracle {c['K'].shape[0]}"
+    L = ring + wl.text_len
     want_rows = np.empty(rows, dtype=np.int64)
     for r in range(rows):
         if r < ring:
             v = r // (T * n)
             t = r % n
             want_rows[r] = idx[(v, int(ex["frame_id"][r]), t)]
-        else:
+        elif r < L:
             want_rows[r] = idx[(-1, -1, r - ring)]
+        else:  # decode tail
+            want_rows[r] = idx[(-2, -1, r - L)]
     # positions: bit-exact
     np.testing.assert_array_equal(ex["pos"], c["pos"][want_rows])
     # contents: the bf16 bit patterns themselves (the oracle holds exact upcasts of them)

@@ -40,7 +40,8 @@ def test_every_declared_symbol_is_exported_and_bound(lib):
 def test_status_codes_match_header():
     text = open(HEADER).read()
     for name in ("FS_OK", "FS_ERR_ARG", "FS_ERR_STATE", "FS_ERR_CUDA", "FS_ERR_DEVICE_TIMEOUT", "FS_ERR_OOM",
-                 "FS_STATE_EXPECT_PREFILL", "FS_STATE_PREFILLED", "FS_STATE_STREAMING", "FS_MAX_VERIFY_TOKENS"):
+                 "FS_ERR_RANGE", "FS_STATE_EXPECT_PREFILL", "FS_STATE_PREFILLED", "FS_STATE_STREAMING",
+                 "FS_MAX_VERIFY_TOKENS", "FS_MAX_TAIL_TOKENS"):
         m = re.search(rf"#define {name}\s+(-?\d+)", text)
         assert m and int(m.group(1)) == getattr(abi, name), name
 
@@ -69,3 +70,6 @@ def test_null_handle_calls_fail_cleanly(lib):
     assert lib.fs_stream_destroy(None) == abi.FS_OK
     assert lib.fs_stream_create(None, 1, 1, 1, 0, 1, 1, 64, 1.0) == abi.FS_ERR_ARG
     assert lib.fs_stream_attend_ext(None, None, None, None, 8, None) == abi.FS_ERR_ARG
+    assert lib.fs_stream_append(None, None, None, 1) == abi.FS_ERR_ARG
+    assert lib.fs_stream_insert_batch(None, 1, None, None) == abi.FS_ERR_ARG
+    assert lib.fs_stream_insert_batch(None, 0, None, None) == abi.FS_ERR_ARG
