@@ -680,6 +680,28 @@ def run_verify(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
+    # The same calls replayed from a CUDA graph (the pages run the decode loop
+    # under CUDA graphs): the device time per call without host dispatch.
+    calls = 16
+    gouts = [torch.empty((nx, wl.H, wl.d), dtype=torch.float32, device=dev) for _ in range(2)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for c in range(calls):
+            b = blocks[c % sets]
+            s.attend_ext(b["Q"], b["K"], b["V"], gouts[c % 2])
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    replays = max(1, args.steps // calls)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(replays):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    graph_ms = max_over_ranks(g0.elapsed_time(g1), world) / (replays * calls)
+    del graph
+    s.sync()
     s.close()
     if world > 1:
         import torch.distributed as dist
@@ -698,6 +720,8 @@ def run_verify(args):
         "warmup": args.warmup,
         "ms_per_step": round(ms, 5),
         "us_per_verify_call": round(ms * 1e3, 2),
+        "us_per_verify_call_graph": round(graph_ms * 1e3, 2),
+        "tflops_graph": round(fl / (graph_ms * 1e-3) / 1e12, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,

@@ -119,6 +119,7 @@ class Stream:
         _check(lib.fs_stream_create(ctypes.byref(h), views, frames, tok_per_frame, text_len, H, Hkv, d,
                                     float(rope_base)))
         self._lib, self.handle = lib, h
+        self._bound = None  # the cudaStream_t last passed to fs_stream_set_stream
         self.views, self.frames, self.tok_per_frame, self.text_len = views, frames, tok_per_frame, text_len
         self.H, self.Hkv, self.d = H, Hkv, d
 
@@ -136,8 +137,10 @@ class Stream:
     def _bind_stream(self):
         import torch
 
-        _check(self._lib.fs_stream_set_stream(self.handle, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)),
-               self.handle)
+        cur = torch.cuda.current_stream().cuda_stream
+        if cur != self._bound:
+            _check(self._lib.fs_stream_set_stream(self.handle, ctypes.c_void_p(cur)), self.handle)
+            self._bound = cur
 
     def info(self) -> fs_stream_info_t:
         i = fs_stream_info_t()
@@ -212,9 +215,8 @@ def insert_batch(streams, K_list, V_list):
     if not (n == len(K_list) == len(V_list)) or n == 0:
         raise ValueError("need one K and one V per stream")
     lib = load()
-    cur = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for s in streams:
-        _check(lib.fs_stream_set_stream(s.handle, cur), s.handle)
+        s._bind_stream()
     hs = (_P * n)(*[s.handle.value for s in streams])
     ks = (_P * n)(*[_ptr(k).value for k in K_list])
     vs = (_P * n)(*[_ptr(v).value for v in V_list])

@@ -1,6 +1,7 @@
 // fs_internal.cuh -- parameters shared by the host side of the library and its
 // kernels, and the position arithmetic of the view-major window.
 #pragma once
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <utility>
@@ -14,6 +15,7 @@ constexpr int kMaxKeyTiles = 2048;      // key rows per kv head <= 2048 * 128
 constexpr int kMaxVerify = 256;         // scratch rows for a drafted block (FS_MAX_VERIFY_TOKENS)
 constexpr int kMaxTail = 1024;          // persisted decode-tail rows (FS_MAX_TAIL_TOKENS)
 constexpr int kMaxInsertBatch = 40;     // layers one kv_stream_insert launch covers
+constexpr int kMaxVerifySplits = 16;    // key splits per kv head of a verify_attn launch (its cluster size)
 constexpr unsigned kErrTimeout = 1u;    // device error word bits
 constexpr unsigned kErrBadLaunch = 2u;
 constexpr unsigned kErrRange = 4u;      // an fp16 operand would overflow (|x| > 65504) or is NaN
@@ -137,6 +139,25 @@ struct InsertParams {
     InsertLayer layer[kMaxInsertBatch];
 };
 
+// A drafted block's attention in one launch (kernel verify_attn).
+struct VerifyParams {
+    WindowShape w;
+    int key_rows;           // L + tail + n_x: cached rows, then the block's rows
+    int row_block;          // L + tail: physical row (= position) of the block's first token
+    int n_x;                // block tokens (n_x * G <= 128)
+    int Hkv, G, H, d, rows_cap;
+    int splits;             // key splits per kv head = cluster size (grid = Hkv * splits)
+    float q_scale;          // log2(e) / sqrt(d)
+    const float2* rope;     // [rope_rows][d/2] (cos, sin)
+    const RingState* state; // angle offset k * n
+    const uint16_t* Q_x;    // [n_x][H][d] bf16
+    const uint16_t* K_x;    // [n_x][Hkv][d] bf16
+    const uint16_t* V_x;
+    float* out;             // [n_x][H][d] fp32
+    unsigned* err;
+    unsigned long long wait_limit_ns;
+};
+
 // Launches `kernel` with programmatic stream serialisation: its launch and set-up
 // may overlap the end of the previous kernel on the stream; the kernel itself
 // calls grid_dependency_wait() before touching memory that kernel may use.
@@ -165,6 +186,22 @@ cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Raises `Kernel`'s dynamic shared-memory limit to `bytes` once per device (the
+// attribute is per device and per function; the first launch on each device
+// sets it, later launches skip the call).
+template <auto Kernel>
+cudaError_t ensure_smem_attr(int bytes) {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(bytes, std::memory_order_release);
+    return e;
+}
+
 // Launchers (defined in the .cu files); all enqueue on `stream` and return the
 // launch's cudaError_t.
 // kv_stream_insert: new K/V into the bf16 cache, and every processed row's rotated
@@ -177,6 +214,10 @@ cudaError_t launch_kv_stream_insert(const InsertParams& p, cudaStream_t stream);
 cudaError_t launch_stream_attn(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkh,
                                const CUtensorMap& tkl, const CUtensorMap& tv16, cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
+// verify_attn over the operand cache; tkh / tkl: K hi / lo maps with 64-row
+// boxes, tv: V map with {64 columns, 128 rows} boxes (128-byte swizzle).
+cudaError_t launch_verify_attn(const VerifyParams& p, const CUtensorMap& tkh, const CUtensorMap& tkl,
+                               const CUtensorMap& tv, cudaStream_t stream);
 cudaError_t launch_positions(const WindowShape& w, const RingState* state, int rows, int* pos_out,
                              cudaStream_t stream);
 cudaError_t launch_wait_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);

@@ -54,6 +54,7 @@ struct fs_stream {
     cudaStream_t copy_in = nullptr, copy_out = nullptr;         // host-path copy streams
     cudaEvent_t ev_in = nullptr, ev_done = nullptr, ev_out = nullptr;
     CUtensorMap tmap_kh2, tmap_kl2, tmap_v16h;  // fp16 operands, one CTA's half tile (attention loads)
+    CUtensorMap tmap_v1;    // fp16 V, {64 columns, 128 rows} boxes (drafted-block verify)
     unsigned long long wait_limit_ns = 2000000000ull;
     long long cache_bytes = 0;
     long long launches = 0;
@@ -351,6 +352,37 @@ int check_block_args(fs_stream_t s, const void* Q_x, const void* K_x, const void
     return FS_OK;
 }
 
+// A drafted block whose queries fit one 128-row tile per kv head goes through
+// verify_attn (one launch: block rotation, split-KV attention, in-kernel
+// merge); longer blocks through kv_stream_insert + stream_attn (+ combine).
+int verify_small(fs_stream_t s, const void* Q_x, const void* K_x, const void* V_x, int n_x, void* out) {
+    fs::VerifyParams p;
+    std::memset(&p, 0, sizeof p);
+    p.w = shape_of(s);
+    p.row_block = s->L + s->tail;
+    p.key_rows = p.row_block + n_x;
+    p.n_x = n_x;
+    p.Hkv = s->Hkv;
+    p.G = s->G;
+    p.H = s->H;
+    p.d = s->d;
+    p.rows_cap = s->rows_cap;
+    const int nkt = (p.key_rows + fs::kTileRows - 1) / fs::kTileRows;
+    p.splits = std::min(fs::kMaxVerifySplits, nkt);
+    p.q_scale = float(1.4426950408889634 / std::sqrt(double(s->d)));
+    p.rope = s->rope;
+    p.state = s->dstate;
+    p.Q_x = static_cast<const uint16_t*>(Q_x);
+    p.K_x = static_cast<const uint16_t*>(K_x);
+    p.V_x = static_cast<const uint16_t*>(V_x);
+    p.out = static_cast<float*>(out);
+    p.err = s->err;
+    p.wait_limit_ns = s->wait_limit_ns;
+    FS_CUDA(s, fs::launch_verify_attn(p, s->tmap_kh2, s->tmap_kl2, s->tmap_v1, s->stream));
+    s->launches += 1;
+    return FS_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -455,6 +487,8 @@ int fs_stream_create(fs_stream_t* out, int views, int frames, int tok_per_frame,
     if (!rc) rc = make_map(nullptr, &s->tmap_v16h, s->V16, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
                            fs::kTileRows, 1, f16, uint32_t(d / 2),
                            d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+    if (!rc) rc = make_map(nullptr, &s->tmap_v1, s->V16, d, s->rows_cap, Hkv, row_bytes, row_bytes * s->rows_cap,
+                           fs::kTileRows, 1, f16, 64u, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return bail(rc);
     *out = s;
     return FS_OK;
@@ -559,6 +593,7 @@ int fs_stream_attend_ext(fs_stream_t s, const void* Q_x, const void* K_x, const 
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
     int rc = check_block_args(s, Q_x, K_x, V_x, n_x, out);
     if (rc) return rc;
+    if (n_x * s->G <= fs::kTileRows) return verify_small(s, Q_x, K_x, V_x, n_x, out);
     CUtensorMap tq;
     rc = make_query_map(s, &tq, Q_x, n_x);
     if (rc) return rc;

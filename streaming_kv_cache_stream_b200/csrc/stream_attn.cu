@@ -235,15 +235,6 @@ __device__ __forceinline__ bool vote_all_ok(uint32_t id, uint32_t threads, bool 
     return res != 0;
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-
 // Smallest visible key tile index >= j (the caller knows one exists).
 __device__ __forceinline__ int next_visible(const uint32_t* vis, int j) {
     int w = j >> 5;
@@ -838,13 +829,8 @@ template <int D>
 cudaError_t launch_d(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkh, const CUtensorMap& tkl,
                      const CUtensorMap& tv16, cudaStream_t stream) {
     const size_t smem = stream_attn_smem_bytes(D);
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(stream_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(smem));
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    cudaError_t e = ensure_smem_attr<stream_attn_kernel<D>>(int(smem));
+    if (e != cudaSuccess) return e;
     const int units = (p.q_tiles + 3) / 4;
     const unsigned grid = unsigned(2 * units * p.Hkv * p.splits);
     return launch_overlapped(stream_attn_kernel<D>, dim3(grid), dim3(kThreads), smem, stream, p, tq, tkh, tkl, tv16);

@@ -286,3 +286,80 @@ def test_out_of_range_input_is_reported():
     s.insert(to_dev(window_inputs(1, 0, 1)["K"]), to_dev(window_inputs(1, 0, 1)["V"]))
     s.sync()
     s.close()
+
+
+@pytest.mark.parametrize("shape,nxs", [
+    ((4, 4, 64, 32, 32, 8, 128), (1, 8, 31, 32, 33)),   # G = 4: one query tile up to 32 tokens, 33 takes the long path
+    ((2, 3, 50, 7, 16, 2, 64), (1, 16, 17)),            # G = 8, d = 64
+    ((1, 2, 100, 0, 4, 4, 128), (5, 128, 129)),         # G = 1, no text
+])
+def test_verify_block_sizes_against_oracle(shape, nxs):
+    """Drafted blocks on both sides of the one-tile limit (n_x * G <= 128 runs
+    the single-launch verify kernel), after a window step and with a decode
+    tail, against the oracle."""
+    import torch
+
+    V_, T, n, X, H, Hkv, d = shape
+    wl = Workload("verify-sizes", V_, T, n, X, H=H, Hkv=Hkv, d=d, steps=1)
+    s = make_stream(wl)
+    orc = make_oracle(wl)
+    rng = np.random.default_rng(sum(shape))
+    for k in range(2):
+        N = wl.tokens(k)
+        b = {"Q": _bits(rng, N, H, d), "K": _bits(rng, N, Hkv, d), "V": _bits(rng, N, Hkv, d)}
+        s.insert(to_dev(b["K"]), to_dev(b["V"]))
+        s.attend(to_dev(b["Q"]), out_like(to_dev(b["Q"])))
+        (orc.prefill if k == 0 else orc.step)(f64(b["Q"]), f64(b["K"]), f64(b["V"]))
+    for with_tail in (False, True):
+        if with_tail:
+            acc = {"K": _bits(rng, 11, Hkv, d), "V": _bits(rng, 11, Hkv, d)}
+            s.append(to_dev(acc["K"]), to_dev(acc["V"]))
+            orc.append(f64(acc["K"]), f64(acc["V"]))
+        for nx in nxs:
+            bx = {"Q": _bits(rng, nx, H, d), "K": _bits(rng, nx, Hkv, d), "V": _bits(rng, nx, Hkv, d)}
+            Qx = to_dev(bx["Q"])
+            ox = out_like(Qx)
+            s.attend_ext(Qx, to_dev(bx["K"]), to_dev(bx["V"]), ox)
+            torch.cuda.synchronize()
+            compare(from_dev(ox), orc.verify(f64(bx["Q"]), f64(bx["K"]), f64(bx["V"])),
+                    f"{shape} n_x={nx} tail={with_tail}")
+    s.sync()
+    check_cache_bitexact(s, orc, wl)
+    s.close()
+
+
+def test_verify_calls_replayed_from_a_cuda_graph():
+    """Verify calls captured in a CUDA graph and replayed give the eager
+    results bit for bit (no launch parameter depends on host state that the
+    replay would freeze; the merge counters reset themselves)."""
+    import torch
+
+    wl = WORKLOADS[5]
+    s = make_stream(wl)
+    for k in range(wl.steps + 1):
+        inp = window_inputs(5, 0, k)
+        Q, K, V = (to_dev(inp[x]) for x in ("Q", "K", "V"))
+        s.insert(K, V)
+        s.attend(Q, out_like(Q))
+    blocks = [{x: to_dev(verify_inputs(5, c)[x]) for x in ("Q", "K", "V")} for c in range(3)]
+    eager = []
+    for b in blocks:
+        o = out_like(b["Q"])
+        s.attend_ext(b["Q"], b["K"], b["V"], o)
+        eager.append(o)
+    torch.cuda.synchronize()
+    outs = [out_like(b["Q"]) for b in blocks]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for b, o in zip(blocks, outs):
+            s.attend_ext(b["Q"], b["K"], b["V"], o)
+    for _ in range(3):
+        for o in outs:
+            o.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for o, e in zip(outs, eager):
+            assert torch.equal(o, e)
+    del g
+    s.sync()
+    s.close()
