@@ -7,6 +7,7 @@ from .stream_oracle import (  # noqa: F401
     StreamOracle,
     ViewMajorWindow,
     bf16_bits_to_f64,
+    frame_attention,
     masked_attention,
     rope_frequencies,
     rope_rotate,

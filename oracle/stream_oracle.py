@@ -27,6 +27,12 @@ What it computes, and where the pages define it (FlashDrive, arXiv 2608.12932):
 * Speculative verification of a drafted 8-token block in one forward --
   FlashDrive README (z-lab/flashdrive), "Speculative reasoning (DFlash)";
   technical summary (gist.science), Methodology 2.
+* Encode only the newest frame: a window step runs the vision encoder on each
+  view's newest frame and reuses the rest -- technical summary (gist.science),
+  Methodology 1, "Algorithmic Shortcut"; paper review (romaanj.github.io),
+  Figure 2 caption. Within the encoder, a frame's tokens attend to each other
+  (reading: plain bidirectional softmax attention per view, no positional
+  rotation, 1/sqrt(d); the pages name no encoder internals).
 * Accepted draft tokens become context for the next drafted block (the
   decode stage produces reasoning tokens after the prompt; the drafter's
   blocks of 8 are accepted 5.6 tokens at a time on average) -- technical
@@ -79,6 +85,7 @@ __all__ = [
     "visible_mask",
     "kv_head_of",
     "score_scale",
+    "frame_attention",
 ]
 
 
@@ -179,6 +186,36 @@ def masked_attention(Q: np.ndarray, qpos: np.ndarray, K: np.ndarray, V: np.ndarr
         p = np.exp(s)
         p /= p.sum(axis=1, keepdims=True)
         out[:, h, :] = p @ V[:, kv, :]
+    return out
+
+
+def frame_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, views: int, n: int) -> np.ndarray:
+    """Encoder attention over the newest frame of each view, in float64.
+
+    Q [views*n, H, d], K and V [views*n, Hkv, d], tokens view-major (view v's
+    frame is rows v*n .. v*n + n - 1). Every token of view v attends to every
+    token of view v's frame (bidirectional, no mask inside the frame) and to
+    nothing else; no rotation; scores scaled by 1/sqrt(d); query head h reads
+    kv head h // (H/Hkv). Returns [views*n, H, d].
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    nt, H, d = Q.shape
+    Hkv = K.shape[1]
+    if nt != views * n or K.shape[0] != nt or V.shape[0] != nt or H % Hkv:
+        raise ValueError("bad frame shapes")
+    out = np.empty((nt, H, d), dtype=np.float64)
+    scale = score_scale(d)
+    for v in range(views):
+        rows = slice(v * n, (v + 1) * n)
+        for h in range(H):
+            kv = kv_head_of(h, H, Hkv)
+            s = (Q[rows, h, :] @ K[rows, kv, :].T) * scale
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p /= p.sum(axis=1, keepdims=True)
+            out[rows, h, :] = p @ V[rows, kv, :]
     return out
 
 

@@ -621,3 +621,95 @@ def test_planted_tail_kept_across_steps(monkeypatch):
         orig(self, K_new, V_new)
         self.tail_K, self.tail_V = keep
     _expect_caught(monkeypatch, (ViewMajorWindow, "step"), bad, TAIL_PINS)
+
+
+# ------------------------------------------------ encoder attention (newest frame)
+
+def _brute_frame(Q, K, V, views, n):
+    """Scalar Python: each view's frame tokens attend to each other, nothing else."""
+    nt, H, d = Q.shape
+    Hkv = K.shape[1]
+    G = H // Hkv
+    out = np.zeros((nt, H, d))
+    for v in range(views):
+        for a in range(v * n, (v + 1) * n):
+            for h in range(H):
+                kv = h // G
+                sc = [sum(float(Q[a, h, i]) * float(K[b, kv, i]) for i in range(d)) / math.sqrt(d)
+                      for b in range(v * n, (v + 1) * n)]
+                mx = max(sc)
+                w = [math.exp(x - mx) for x in sc]
+                tot = sum(w)
+                for i in range(d):
+                    out[a, h, i] = sum(w[j] * float(V[v * n + j, kv, i]) for j in range(n)) / tot
+    return out
+
+
+def pin_frame_brute(views=2, n=5, H=4, Hkv=2, d=8, seed=31):
+    rng = np.random.default_rng(seed)
+    Q = bf16_bits_to_f64(_rand(rng, views * n, H, d))
+    K = bf16_bits_to_f64(_rand(rng, views * n, Hkv, d))
+    V = bf16_bits_to_f64(_rand(rng, views * n, Hkv, d))
+    np.testing.assert_allclose(so.frame_attention(Q, K, V, views, n), _brute_frame(Q, K, V, views, n),
+                               rtol=0, atol=1e-12)
+
+
+def pin_frame_is_sdpa_per_view(views=3, n=17, H=8, Hkv=2, d=16, seed=32):
+    """Each view's frame is torch SDPA (float64, no mask, GQA) over that frame alone."""
+    rng = np.random.default_rng(seed)
+    Q = bf16_bits_to_f64(_rand(rng, views * n, H, d))
+    K = bf16_bits_to_f64(_rand(rng, views * n, Hkv, d))
+    V = bf16_bits_to_f64(_rand(rng, views * n, Hkv, d))
+    got = so.frame_attention(Q, K, V, views, n)
+    for v in range(views):
+        r = slice(v * n, (v + 1) * n)
+        q = torch.tensor(Q[r]).permute(1, 0, 2)[None]
+        k = torch.tensor(K[r]).permute(1, 0, 2)[None]
+        vv = torch.tensor(V[r]).permute(1, 0, 2)[None]
+        o = torch.nn.functional.scaled_dot_product_attention(q, k, vv, is_causal=False, enable_gqa=True)
+        np.testing.assert_allclose(got[r], o[0].permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+
+
+def pin_frame_permutation_and_isolation(views=2, n=9, H=2, Hkv=1, d=8, seed=33):
+    """Bidirectional with no positions: permuting a frame's tokens permutes its
+    output rows; changing one view's tokens leaves the other views' output alone."""
+    rng = np.random.default_rng(seed)
+    Q = bf16_bits_to_f64(_rand(rng, views * n, H, d))
+    K = bf16_bits_to_f64(_rand(rng, views * n, Hkv, d))
+    V = bf16_bits_to_f64(_rand(rng, views * n, Hkv, d))
+    base = so.frame_attention(Q, K, V, views, n)
+    perm = np.concatenate([rng.permutation(n) + v * n for v in range(views)])
+    got = so.frame_attention(Q[perm], K[perm], V[perm], views, n)
+    np.testing.assert_allclose(got, base[perm], rtol=0, atol=1e-12)
+    K2, V2 = K.copy(), V.copy()
+    K2[n:] = bf16_bits_to_f64(_rand(rng, (views - 1) * n, Hkv, d))
+    V2[n:] = bf16_bits_to_f64(_rand(rng, (views - 1) * n, Hkv, d))
+    np.testing.assert_array_equal(so.frame_attention(Q, K2, V2, views, n)[:n], base[:n])
+
+
+FRAME_PINS = [pin_frame_brute, pin_frame_is_sdpa_per_view, pin_frame_permutation_and_isolation]
+
+
+def test_frame_attention_pins():
+    for pin in FRAME_PINS:
+        pin()
+
+
+def test_planted_frame_causal_mask(monkeypatch):
+    """A causal mask inside the frame (the streaming path's habit) is caught."""
+    def bad(Q, K, V, views, n):
+        Q = np.asarray(Q, dtype=np.float64)
+        out = np.empty(Q.shape)
+        for v in range(views):
+            r = slice(v * n, (v + 1) * n)
+            pos = np.arange(n)
+            out[r] = so.masked_attention(Q[r], pos, K[r], V[r], pos, 1.0)  # base 1.0: angle 0 only at pos 0
+        return out
+    _expect_caught(monkeypatch, (so, "frame_attention"), bad, FRAME_PINS)
+
+
+def test_planted_frame_across_views(monkeypatch):
+    """Attention that leaks across views is caught."""
+    def bad(Q, K, V, views, n):
+        return so.masked_attention(Q, np.zeros(len(Q)), K, V, np.zeros(len(K)), 10000.0)
+    _expect_caught(monkeypatch, (so, "frame_attention"), bad, FRAME_PINS)
