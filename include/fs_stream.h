@@ -233,6 +233,26 @@ int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x,
                                 int n_x, void* out);
 
 /*
+ * fs_frame_attend -- the vision encoder's attention over the newest frame of
+ * each view (FlashDrive technical summary, Methodology 1, "Algorithmic
+ * Shortcut": a window step encodes only each camera's newest frame and reuses
+ * the rest). For view v, token t of its frame attends to every token of the
+ * same frame -- bidirectional, nothing of other views, no rotation (the pages
+ * name no encoder internals; plain softmax attention is the reading taken),
+ * scores scaled by 1/sqrt(d), query head h reading kv head h / (H/Hkv).
+ *   Q [views * tok_per_frame][H][d] bf16, K and V [views * tok_per_frame][Hkv][d]
+ *   bf16 (token t of view v at row v * tok_per_frame + t, device);
+ *   out [views * tok_per_frame][H][d] fp32. views and tok_per_frame are the
+ *   handle's; H, Hkv, d are the encoder's (H % Hkv == 0, 128 % (H/Hkv) == 0,
+ *   d in {64, 128}). The handle supplies the stream and the error word only;
+ *   its cache is not touched and its state does not matter.
+ * Range: |V| <= 65504 (V is converted to fp16 for P V); checked, reported by
+ * fs_stream_sync as FS_ERR_RANGE.
+ * Errors: FS_ERR_ARG, FS_ERR_CUDA.
+ */
+int fs_frame_attend(fs_stream_t s, const void* Q, const void* K, const void* V, int H, int Hkv, int d, void* out);
+
+/*
  * fs_stream_step_host -- one insert + attend with HOST buffers: copies K_new,
  * V_new and Q (bf16) to the device (staging buffers owned by the handle), runs
  * fs_stream_insert and fs_stream_attend on the handle's stream, and copies out

@@ -50,6 +50,7 @@ SIGNATURES = {
     "fs_stream_attend": (_I, [_P, _P, _P]),
     "fs_stream_attend_ext": (_I, [_P, _P, _P, _P, _I, _P]),
     "fs_stream_attend_ext_static": (_I, [_P, _P, _P, _P, _I, _P]),
+    "fs_frame_attend": (_I, [_P, _P, _P, _P, _I, _I, _I, _P]),
     "fs_stream_step_host": (_I, [_P, _P, _P, _P, _P]),
     "fs_stream_sync": (_I, [_P]),
     "fs_stream_info": (_I, [_P, ctypes.POINTER(fs_stream_info_t)]),
@@ -174,6 +175,13 @@ class Stream:
         self._bind_stream()
         _check(self._lib.fs_stream_attend_ext_static(self.handle, _ptr(Q_x), _ptr(K_x), _ptr(V_x),
                                                      int(Q_x.shape[0]), _ptr(out, "float32")), self.handle)
+
+    def frame_attend(self, Q, K, V, out):
+        """Encoder attention over each view's newest frame: Q [views*n, H, d],
+        K/V [views*n, Hkv, d] bf16 -> out fp32 [views*n, H, d]."""
+        self._bind_stream()
+        _check(self._lib.fs_frame_attend(self.handle, _ptr(Q), _ptr(K), _ptr(V), int(Q.shape[1]), int(K.shape[1]),
+                                         int(Q.shape[2]), _ptr(out, "float32")), self.handle)
 
     def step_host(self, K_new_h, V_new_h, Q_h, out_h):
         """Host-buffer step: numpy/torch CPU buffers (pinned for asynchrony)."""

@@ -186,6 +186,20 @@ cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The vision encoder's attention over each view's newest frame (kernel frame_attn).
+struct FrameParams {
+    int views, n;           // views, tokens per frame; token t of view v is row v * n + t
+    int H, Hkv, G, d;
+    int q_tiles;            // ceil(n * G / 128) query tiles per (view, kv head)
+    float q_scale;          // log2(e) / sqrt(d)
+    const uint16_t* Q;      // [views * n][H][d] bf16
+    const uint16_t* K;      // [views * n][Hkv][d] bf16
+    const uint16_t* V;
+    float* out;             // [views * n][H][d] fp32
+    unsigned* err;
+    unsigned long long wait_limit_ns;
+};
+
 // Raises `Kernel`'s dynamic shared-memory limit to `bytes` once per device (the
 // attribute is per device and per function; the first launch on each device
 // sets it, later launches skip the call).
@@ -218,6 +232,7 @@ cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
 // boxes, tv: V map with {64 columns, 128 rows} boxes (128-byte swizzle).
 cudaError_t launch_verify_attn(const VerifyParams& p, const CUtensorMap& tkh, const CUtensorMap& tkl,
                                const CUtensorMap& tv, cudaStream_t stream);
+cudaError_t launch_frame_attn(const FrameParams& p, cudaStream_t stream);
 cudaError_t launch_positions(const WindowShape& w, const RingState* state, int rows, int* pos_out,
                              cudaStream_t stream);
 cudaError_t launch_wait_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);

@@ -655,6 +655,37 @@ int fs_stream_attend_ext_static(fs_stream_t s, const void* Q_x, const void* K_x,
 // copy-out stream returns the output. Consecutive calls on different handles
 // (layers) therefore overlap one layer's upload, another's kernels and a
 // third's download; fs_stream_sync waits for all three streams.
+int fs_frame_attend(fs_stream_t s, const void* Q, const void* K, const void* V, int H, int Hkv, int d, void* out) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (!Q || !K || !V || !out) return fail(s, FS_ERR_ARG, "NULL tensor pointer");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out))
+        return fail(s, FS_ERR_ARG, "pointers must be 16-byte aligned");
+    if (out == Q || out == K || out == V) return fail(s, FS_ERR_ARG, "out must not alias an input");
+    if (H < 1 || Hkv < 1 || H % Hkv) return fail(s, FS_ERR_ARG, "need H, Hkv >= 1 and H %% Hkv == 0");
+    const int G = H / Hkv;
+    if (fs::kTileRows % G) return fail(s, FS_ERR_ARG, "H/Hkv must divide 128 (got %d)", G);
+    if (d != 64 && d != 128) return fail(s, FS_ERR_ARG, "head dim must be 64 or 128 (got %d)", d);
+    fs::FrameParams p;
+    std::memset(&p, 0, sizeof p);
+    p.views = s->V;
+    p.n = s->n;
+    p.H = H;
+    p.Hkv = Hkv;
+    p.G = G;
+    p.d = d;
+    p.q_tiles = (s->n * G + fs::kTileRows - 1) / fs::kTileRows;
+    p.q_scale = float(1.4426950408889634 / std::sqrt(double(d)));
+    p.Q = static_cast<const uint16_t*>(Q);
+    p.K = static_cast<const uint16_t*>(K);
+    p.V = static_cast<const uint16_t*>(V);
+    p.out = static_cast<float*>(out);
+    p.err = s->err;
+    p.wait_limit_ns = s->wait_limit_ns;
+    FS_CUDA(s, fs::launch_frame_attn(p, s->stream));
+    s->launches += 1;
+    return FS_OK;
+}
+
 int fs_stream_step_host(fs_stream_t s, const void* K_new_h, const void* V_new_h, const void* Q_h, void* out_h) {
     if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
     if (!K_new_h || !V_new_h || !Q_h || !out_h) return fail(s, FS_ERR_ARG, "NULL host pointer");

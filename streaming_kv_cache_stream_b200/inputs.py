@@ -7,7 +7,8 @@ so both the CUDA path and the CPU oracle may take their inputs from it.
 Every tensor is drawn from numpy's PCG64 seeded with
 ``SeedSequence([workload, layer, step, tensor, call])`` as float32 standard
 normals, multiplied by the workload's scale, then rounded to bf16
-(round-to-nearest-even). Tensor ids: Q = 0, K = 1, V = 2, outlier-row choice = 3.
+(round-to-nearest-even). Tensor ids: Q = 0, K = 1, V = 2, outlier-row choice = 3;
+the encoder attention's Q, K, V = 10, 11, 12.
 Step 0 is the prefill window (the stream's first call); steps 1.. are window
 steps; ``call`` numbers the verify calls.
 
@@ -21,6 +22,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 Q_ID, K_ID, V_ID, OUTLIER_ID = 0, 1, 2, 3
+FRAME_Q_ID, FRAME_K_ID, FRAME_V_ID = 10, 11, 12  # encoder attention over the newest frames
 
 
 @dataclass(frozen=True)
@@ -133,4 +135,23 @@ def verify_inputs(wid: int, call: int, layer: int = 0) -> dict:
         Q=draw_bf16(wid, layer, step, Q_ID, call + 1, (nx, wl.H, wl.d)),
         K=draw_bf16(wid, layer, step, K_ID, call + 1, (nx, wl.Hkv, wl.d)),
         V=draw_bf16(wid, layer, step, V_ID, call + 1, (nx, wl.Hkv, wl.d)),
+    )
+
+
+# Head layout of the vision encoder's attention (the pages give none): 16 heads
+# of 64, multi-head (no grouping), a ViT-style encoder layer.
+FRAME_HEADS = dict(H=16, Hkv=16, d=64)
+
+
+def frame_inputs(wid: int, layer: int, step: int, H: int = FRAME_HEADS["H"], Hkv: int = FRAME_HEADS["Hkv"],
+                 d: int = FRAME_HEADS["d"]) -> dict:
+    """The newest frame of every view, as the encoder's attention sees it:
+    Q [views*n, H, d], K and V [views*n, Hkv, d] bf16 bits, ~N(0,1), token t of
+    view v at row v*n + t (n = the workload's tokens per frame)."""
+    wl = WORKLOADS[wid]
+    rows = wl.views * wl.tok_per_frame
+    return dict(
+        Q=draw_bf16(wid, layer, step, FRAME_Q_ID, 0, (rows, H, d)),
+        K=draw_bf16(wid, layer, step, FRAME_K_ID, 0, (rows, Hkv, d)),
+        V=draw_bf16(wid, layer, step, FRAME_V_ID, 0, (rows, Hkv, d)),
     )
