@@ -7,7 +7,9 @@ from .stream_oracle import (  # noqa: F401
     StreamOracle,
     ViewMajorWindow,
     bf16_bits_to_f64,
+    bf16_round,
     frame_attention,
+    project_kv,
     masked_attention,
     rope_frequencies,
     rope_rotate,

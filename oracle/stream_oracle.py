@@ -33,6 +33,12 @@ What it computes, and where the pages define it (FlashDrive, arXiv 2608.12932):
   Figure 2 caption. Within the encoder, a frame's tokens attend to each other
   (reading: plain bidirectional softmax attention per view, no positional
   rotation, 1/sqrt(d); the pages name no encoder internals).
+* Fused projections: the Q, K, V projections are merged into one kernel --
+  README (z-lab/flashdrive), "System optimizations"; technical summary,
+  System Optimizations, "Kernel Fusion". Here the K/V projection of a step's
+  hidden states is K = X W_k^T, V = X W_v^T, each output rounded once to bf16
+  (round to nearest, ties to even) before it is cached (reading: the cache
+  holds bf16, the pages give no other precision).
 * Accepted draft tokens become context for the next drafted block (the
   decode stage produces reasoning tokens after the prompt; the drafter's
   blocks of 8 are accepted 5.6 tokens at a time on average) -- technical
@@ -86,6 +92,8 @@ __all__ = [
     "kv_head_of",
     "score_scale",
     "frame_attention",
+    "bf16_round",
+    "project_kv",
 ]
 
 
@@ -187,6 +195,34 @@ def masked_attention(Q: np.ndarray, qpos: np.ndarray, K: np.ndarray, V: np.ndarr
         p /= p.sum(axis=1, keepdims=True)
         out[:, h, :] = p @ V[:, kv, :]
     return out
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value (8 significant bits), ties
+    to even, directly (no intermediate float32 rounding). Finite inputs within
+    the bf16 range; returns float64."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    e = np.floor(np.log2(np.abs(x[nz])))
+    e = np.maximum(e, -126.0)  # below the smallest normal the spacing stays 2^-133
+    ulp = np.exp2(e - 7.0)
+    out[nz] = np.rint(x[nz] / ulp) * ulp  # rint: nearest, ties to even
+    return out
+
+
+def project_kv(X: np.ndarray, W: np.ndarray, Hkv: int, d: int):
+    """K/V projection of hidden states: X [N, d_model] (bf16 values as float64),
+    W [2*Hkv*d, d_model] (rows 0 .. Hkv*d-1 project K, the rest V, as in a
+    linear layer's weight). Returns K, V [N, Hkv, d]: X W^T in float64, each
+    element rounded once to bf16."""
+    X = np.asarray(X, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    if W.shape != (2 * Hkv * d, X.shape[1]):
+        raise ValueError("W must be [2*Hkv*d, d_model]")
+    Y = bf16_round(X @ W.T)
+    n = X.shape[0]
+    return Y[:, :Hkv * d].reshape(n, Hkv, d), Y[:, Hkv * d:].reshape(n, Hkv, d)
 
 
 def frame_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, views: int, n: int) -> np.ndarray:

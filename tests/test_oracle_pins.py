@@ -713,3 +713,69 @@ def test_planted_frame_across_views(monkeypatch):
     def bad(Q, K, V, views, n):
         return so.masked_attention(Q, np.zeros(len(Q)), K, V, np.zeros(len(K)), 10000.0)
     _expect_caught(monkeypatch, (so, "frame_attention"), bad, FRAME_PINS)
+
+
+# ------------------------------------------------------------- K/V projection
+
+def pin_bf16_round_definition(seed=41):
+    """bf16_round returns a bf16 value (float32 with zero low 16 bits) at least as
+    close as both neighbours, ties going to the even significand."""
+    rng = np.random.default_rng(seed)
+    x = np.concatenate([rng.standard_normal(2000) * np.exp2(rng.integers(-20, 20, 2000)),
+                        np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 3.0, 0.0,
+                                  1.0 + 2 ** -8 + 2 ** -30])])  # just above a tie: nearest is 1 + 2^-7
+    b = so.bf16_round(x)
+    b32 = b.astype(np.float32)
+    assert np.array_equal(b32.astype(np.float64), b)
+    assert not np.any(b32.view(np.uint32) & np.uint32(0xFFFF))
+    for xi, bi in zip(x, b):
+        if xi == 0:
+            assert bi == 0
+            continue
+        bits = np.float32(bi).view(np.uint32)
+        up = float(np.uint32(bits + np.uint32(0x10000)).view(np.float32))
+        dn = float(np.uint32(bits - np.uint32(0x10000)).view(np.float32))
+        err = abs(xi - bi)
+        assert err <= abs(xi - up) and err <= abs(xi - dn), (xi, bi)
+        if err == abs(xi - up) or err == abs(xi - dn):  # a tie: the even significand wins
+            assert (bits >> np.uint32(16)) & np.uint32(1) == 0, (xi, bi)
+    np.testing.assert_array_equal(so.bf16_round(np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8])), [1.0, 1.0 + 2 ** -6])
+
+
+def pin_project_kv_brute(n=3, dm=6, Hkv=2, d=4, seed=42):
+    rng = np.random.default_rng(seed)
+    X = bf16_bits_to_f64(_rand(rng, n, dm))
+    W = bf16_bits_to_f64(_rand(rng, 2 * Hkv * d, dm))
+    K, V = so.project_kv(X, W, Hkv, d)
+    for t in range(n):
+        for o in range(2 * Hkv * d):
+            y = 0.0
+            for i in range(dm):
+                y += float(X[t, i]) * float(W[o, i])
+            want = so.bf16_round(np.array([y]))[0]
+            got = K[t, o // d, o % d] if o < Hkv * d else V[t, (o - Hkv * d) // d, o % d]
+            assert got == want, (t, o, got, want)
+
+
+def test_projection_pins():
+    pin_bf16_round_definition()
+    pin_project_kv_brute()
+    pin_project_kv_brute(n=5, dm=16, Hkv=1, d=8, seed=43)
+
+
+def test_planted_projection_transposed(monkeypatch):
+    """Using W's transpose layout (K from columns instead of rows) is caught."""
+    def bad(X, W, Hkv, d):
+        Y = so.bf16_round(np.asarray(X) @ np.asarray(W).reshape(np.asarray(W).shape[1], -1))
+        n = Y.shape[0]
+        return Y[:, :Hkv * d].reshape(n, Hkv, d), Y[:, Hkv * d:].reshape(n, Hkv, d)
+    _expect_caught(monkeypatch, (so, "project_kv"), bad, [pin_project_kv_brute])
+
+
+def test_planted_projection_double_rounding(monkeypatch):
+    """Rounding through float32 first (double rounding) is caught: 1 + 2^-8 + 2^-30
+    becomes the tie 1 + 2^-8 in float32 and then rounds to even (1.0), not to the
+    nearest bf16 value 1 + 2^-7."""
+    _expect_caught(monkeypatch, (so, "bf16_round"),
+                   lambda x: torch.tensor(np.asarray(x, dtype=np.float64)).float().bfloat16().double().numpy(),
+                   [pin_bf16_round_definition])
