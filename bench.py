@@ -420,6 +420,54 @@ def time_frame_attention(wid, calls, dev):
     return us, flops
 
 
+def time_kv_proj(wid, steps, warmup, dev):
+    """fs_stream_insert_proj for every layer of a workload's window step, each
+    layer with its own hidden states and weight (d_model = H*d), launched back
+    to back as a model's step would: CUDA events around each step's calls.
+    Returns (per-call microseconds per step, algorithmic FLOPs per call, bytes
+    per call)."""
+    import numpy as np
+    import torch
+
+    from streaming_kv_cache_stream_b200.abi import Stream
+    from streaming_kv_cache_stream_b200.inputs import WORKLOADS, hidden_inputs, proj_weight
+
+    wl = WORKLOADS[wid]
+    dm = wl.H * wl.d
+    layers = wl.layers
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    hs = [Stream(wl.views, wl.frames, wl.tok_per_frame, wl.text_len, wl.H, wl.Hkv, wl.d, wl.rope_base)
+          for _ in range(layers)]
+    Ws = [to_dev(proj_weight(wid, l, dm)) for l in range(layers)]
+    for l, s in enumerate(hs):
+        s.insert_proj(to_dev(hidden_inputs(wid, l, 0, dm)), Ws[l])
+    Xs = [to_dev(hidden_inputs(wid, l, 1, dm)) for l in range(layers)]
+    stream = torch.cuda.current_stream()
+    ev = []
+    for k in range(warmup + steps):  # fewer steps than the re-base interval (16): no re-rotation pass
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for l, s in enumerate(hs):
+            s.insert_proj(Xs[l], Ws[l])
+        e1.record(stream)
+        if k >= warmup:
+            ev.append((e0, e1))
+    torch.cuda.synchronize()
+    for s in hs:
+        s.sync()
+        s.close()
+    us = [a.elapsed_time(c) * 1e3 / layers for a, c in ev]
+    N, outs = wl.step_tokens, 2 * wl.Hkv * wl.d
+    flops = 2.0 * N * outs * dm
+    nbytes = 2 * (N * dm + outs * dm + N * outs)  # X, W read; K, V written (bf16)
+    del Xs, Ws
+    torch.cuda.empty_cache()
+    return us, flops, nbytes
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -555,6 +603,27 @@ def run_ours(args):
             "l2": "inputs L2-resident (2 MB, as produced by the encoder's previous layer)",
         }
 
+    # ---- the K/V projection fused with the ring insert (one layer's window step)
+    proj = None
+    if rank == 0 and not args.no_wide:
+        pu, pfl, pb = time_kv_proj(wid, 8, 3, dev)
+        pmed = statistics.median(pu)
+        proj = {
+            "kernel": "kv_proj",
+            "bound": "tensor",
+            "shape": f"X [{wl.step_tokens} x {wl.H * wl.d}] x W^T [{wl.H * wl.d} x {2 * wl.Hkv * wl.d}] bf16, "
+                     "epilogue writes the ring slots (bf16) and the rotated fp16 operands",
+            "us_per_call_median": round(pmed, 2),
+            "us_per_call_mean": round(statistics.mean(pu), 2),
+            "algorithmic_gflop_per_call": round(pfl / 1e9, 4),
+            "tflops": round(pfl / (pmed * 1e-6) / 1e12, 2),
+            "frac_of_burst": round(pfl / (pmed * 1e-6) / 1e12 / float(peaks.get("bf16_tflops")), 4),
+            "hbm_floor_us": round(pb / (hbm * 1e3), 2),
+            "l2": "every layer's own X and W (%d MiB per step): no reuse across calls" % (
+                wl.layers * 2 * (wl.step_tokens + 2 * wl.Hkv * wl.d) * wl.H * wl.d // 2 ** 20),
+            "timing": "CUDA events around the %d calls of a step (one per layer, back to back), per call" % wl.layers,
+        }
+
     # ---- end to end through the public C ABI with host buffers
     e2e_steps = max(1, min(args.steps, 5))
     pin = [{x: torch.from_numpy(np.ascontiguousarray(window_inputs(wid, l, 1)[x]).view(np.int16)).pin_memory()
@@ -649,6 +718,7 @@ def run_ours(args):
             },
             "wide_window": wide,
             "frame_encoder": frame,
+            "kv_proj": proj,
             "e2e": {
                 "value": round(world * fl_layer * layers / (e2e_ms * 1e-3) / 1e12, 3),
                 "unit": "TFLOP/s",

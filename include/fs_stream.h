@@ -162,6 +162,22 @@ int fs_stream_insert(fs_stream_t s, const void* K_new, const void* V_new);
 int fs_stream_insert_batch(fs_stream_t* handles, int n, const void* const* K_new, const void* const* V_new);
 
 /*
+ * fs_stream_insert_proj -- fs_stream_insert with the K/V projection fused in
+ * (FlashDrive README, "System optimizations": fused projections; technical
+ * summary, System Optimizations, "Kernel Fusion"). X holds the tokens' hidden
+ * states instead of their K and V:
+ *   X [tokens][d_model] bf16 (device; tokens = L on the prefill, else
+ *   step_tokens, in fs_stream_insert's token order), W [2*Hkv*d][d_model] bf16
+ *   (a linear layer's weight: rows 0 .. Hkv*d-1 give K, the rest V; head h of K
+ *   is rows h*d .. h*d + d - 1). K = X W_k^T and V = X W_v^T are computed on the
+ *   tensor cores in fp32, each element rounded once to bf16 (nearest, ties to
+ *   even) and written into the ring exactly as fs_stream_insert writes K_new /
+ *   V_new, state transitions included. d_model must be a multiple of 8.
+ * Pointers: 16-byte aligned device pointers. Errors: FS_ERR_ARG, FS_ERR_CUDA.
+ */
+int fs_stream_insert_proj(fs_stream_t s, const void* X, const void* W, int d_model);
+
+/*
  * fs_stream_attend -- attention of the last inserted tokens (kernel stream_attn).
  *   State PREFILLED: Q and out are [L][H][d]; query t sits at position t
  *     (plain causal attention over the view-major window).

@@ -47,6 +47,7 @@ SIGNATURES = {
     "fs_stream_insert": (_I, [_P, _P, _P]),
     "fs_stream_insert_batch": (_I, [ctypes.POINTER(_P), _I, ctypes.POINTER(_P), ctypes.POINTER(_P)]),
     "fs_stream_append": (_I, [_P, _P, _P, _I]),
+    "fs_stream_insert_proj": (_I, [_P, _P, _P, _I]),
     "fs_stream_attend": (_I, [_P, _P, _P]),
     "fs_stream_attend_ext": (_I, [_P, _P, _P, _P, _I, _P]),
     "fs_stream_attend_ext_static": (_I, [_P, _P, _P, _P, _I, _P]),
@@ -154,6 +155,13 @@ class Stream:
     def insert(self, K_new, V_new):
         self._bind_stream()
         _check(self._lib.fs_stream_insert(self.handle, _ptr(K_new), _ptr(V_new)), self.handle)
+
+    def insert_proj(self, X, W):
+        """fs_stream_insert_proj: X [tokens, d_model], W [2*Hkv*d, d_model] bf16."""
+        if X.dim() != 2 or W.dim() != 2 or W.shape[1] != X.shape[1] or W.shape[0] != 2 * self.Hkv * self.d:
+            raise ValueError("X must be [tokens, d_model] and W [2*Hkv*d, d_model]")
+        self._bind_stream()
+        _check(self._lib.fs_stream_insert_proj(self.handle, _ptr(X), _ptr(W), int(X.shape[1])), self.handle)
 
     def append(self, K_acc, V_acc):
         """Persist accepted tokens [n, Hkv, d] bf16 at the end of the decode tail."""

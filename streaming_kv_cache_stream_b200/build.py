@@ -19,7 +19,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libfsstream.so")
-SOURCES = ["fs_stream_api.cu", "kv_stream_insert.cu", "stream_attn.cu", "verify_attn.cu", "frame_attn.cu"]
+SOURCES = ["fs_stream_api.cu", "kv_stream_insert.cu", "stream_attn.cu", "verify_attn.cu", "frame_attn.cu", "kv_proj.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr"]
 

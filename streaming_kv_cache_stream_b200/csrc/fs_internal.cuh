@@ -129,7 +129,8 @@ struct InsertLayer {
 
 struct InsertParams {
     WindowShape w;          // window shape (head comes from each layer's state)
-    int mode;               // 0: prefill (row = t), 1: window step, 2: rows [row0, row0 + N) after the text
+    int mode;               // 0: prefill (row = t), 1: window step, 2: rows [row0, row0 + N) after the text,
+                            // 3: re-rotate the window from the cache (state already advanced)
     int N;                  // tokens per layer in K_src / V_src
     int row0;               // mode 2: first physical row written
     int Hkv, d, rows_cap;
@@ -186,6 +187,25 @@ cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The K/V projection of a step's hidden states fused with the ring insert (kernel kv_proj).
+struct ProjParams {
+    WindowShape w;          // window shape (head from the ring state)
+    int mode;               // 0: prefill (token t -> row t), 1: window step
+    int N;                  // tokens (rows of X)
+    int d_model;
+    int Hkv, d, rows_cap;
+    int rebase_every;
+    const float2* rope;
+    uint16_t* K;            // bf16 cache [Hkv][rows_cap][d]
+    uint16_t* V;
+    uint16_t* Kh;           // operands, same layout
+    uint16_t* Kl;
+    uint16_t* V16;
+    RingState* state;
+    unsigned* err;
+    unsigned long long wait_limit_ns;
+};
+
 // The vision encoder's attention over each view's newest frame (kernel frame_attn).
 struct FrameParams {
     int views, n;           // views, tokens per frame; token t of view v is row v * n + t
@@ -233,6 +253,9 @@ cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_verify_attn(const VerifyParams& p, const CUtensorMap& tkh, const CUtensorMap& tkl,
                                const CUtensorMap& tv, cudaStream_t stream);
 cudaError_t launch_frame_attn(const FrameParams& p, cudaStream_t stream);
+// kv_proj over X (tensor map tx: [N][d_model] bf16, box {64, 128}) and W (tw:
+// [2 Hkv d][d_model], box {64, 128}), both 128-byte swizzled.
+cudaError_t launch_kv_proj(const ProjParams& p, const CUtensorMap& tx, const CUtensorMap& tw, cudaStream_t stream);
 cudaError_t launch_positions(const WindowShape& w, const RingState* state, int rows, int* pos_out,
                              cudaStream_t stream);
 cudaError_t launch_wait_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);

@@ -34,6 +34,7 @@ struct fs_stream {
     int state = FS_STATE_EXPECT_PREFILL;
     int head = 0;           // host mirror of the device ring head (sizes, debug export)
     int tail = 0;           // persisted decode-tail tokens after the text
+    int k_host = 0;         // host mirror of the device ring state's step count k
     long long steps = 0;
     std::vector<long long> slot_frame;  // frame id held by each ring slot (same for all views)
     cudaStream_t stream = nullptr;
@@ -264,6 +265,7 @@ void after_window_insert(fs_stream_t s, bool prefill) {
     s->tail = 0;
     if (prefill) {
         s->head = 0;
+        s->k_host = 0;
         s->steps = 0;
         for (int f = 0; f < s->T; ++f) s->slot_frame[f] = f;
         s->state = FS_STATE_PREFILLED;
@@ -271,6 +273,7 @@ void after_window_insert(fs_stream_t s, bool prefill) {
     }
     s->slot_frame[s->head] = (long long)s->T + s->steps;  // the k-th step inserts frame T-1+k
     s->head = (s->head + 1) % s->T;
+    s->k_host = s->k_host + 1 >= s->rebase_every ? 0 : s->k_host + 1;
     s->steps += 1;
     s->state = FS_STATE_STREAMING;
 }
@@ -561,6 +564,53 @@ int fs_stream_insert_batch(fs_stream_t* handles, int n, const void* const* K_new
         s0->launches += 1;
     }
     for (int i = 0; i < n; ++i) after_window_insert(handles[i], prefill);
+    return FS_OK;
+}
+
+int fs_stream_insert_proj(fs_stream_t s, const void* X, const void* W, int d_model) {
+    if (!s) return fail(nullptr, FS_ERR_ARG, "NULL handle");
+    if (!X || !W) return fail(s, FS_ERR_ARG, "X/W is NULL");
+    if (!aligned16(X) || !aligned16(W)) return fail(s, FS_ERR_ARG, "X/W must be 16-byte aligned");
+    if (d_model < 8 || d_model % 8) return fail(s, FS_ERR_ARG, "d_model must be a positive multiple of 8 (got %d)", d_model);
+    const bool prefill = s->state == FS_STATE_EXPECT_PREFILL;
+    const int N = prefill ? s->L : s->step_tokens;
+    const uint64_t row = uint64_t(d_model) * 2;
+    const int outs = 2 * s->Hkv * s->d;
+    CUtensorMap tx, tw;
+    int rc = make_map(s, &tx, X, d_model, N, 1, row, row * N, 128, 1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64);
+    if (!rc) rc = make_map(s, &tw, W, d_model, outs, 1, row, row * outs, 256, 1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64);
+    if (rc) return rc;
+    fs::ProjParams p;
+    std::memset(&p, 0, sizeof p);
+    p.w = shape_of(s);
+    p.mode = prefill ? 0 : 1;
+    p.N = N;
+    p.d_model = d_model;
+    p.Hkv = s->Hkv;
+    p.d = s->d;
+    p.rows_cap = s->rows_cap;
+    p.rebase_every = s->rebase_every;
+    p.rope = s->rope;
+    p.K = s->K_cache;
+    p.V = s->V_cache;
+    p.Kh = s->Kh;
+    p.Kl = s->Kl;
+    p.V16 = s->V16;
+    p.state = s->dstate;
+    p.err = s->err;
+    p.wait_limit_ns = s->wait_limit_ns;
+    FS_CUDA(s, fs::launch_kv_proj(p, tx, tw, s->stream));
+    s->launches += 1;
+    if (!prefill && s->k_host + 1 >= s->rebase_every) {
+        // A re-base step: the projection wrote the new rows' bf16 K/V; the whole
+        // window is re-rotated from the cache at k = 0.
+        InsertParams q = insert_params(s, 3, 0, 0);
+        q.layer[0] = layer_of(s, nullptr, nullptr);
+        q.layers = 1;
+        FS_CUDA(s, fs::launch_kv_stream_insert(q, s->stream));
+        s->launches += 1;
+    }
+    after_window_insert(s, prefill);
     return FS_OK;
 }
 

@@ -23,7 +23,9 @@
 // A launch covers one or more layers (blockIdx.y = layer); each block strides
 // over its layer's rows: the whole window on a prefill or a re-base step, the
 // new rows (each view's new frame and the text) on other steps, and rows
-// [row0, row0 + N) for a decode-tail or drafted block. One thread takes one
+// [row0, row0 + N) for a decode-tail or drafted block, and (mode 3) the whole
+// window from the cache after the fused projection wrote a re-base step's rows.
+// One thread takes one
 // pair of 16-byte chunks (c, c + d/16) of one (row, kv head) -- the
 // rotate-half partners. A row being written this call takes its K/V from the
 // caller's token-major [N][Hkv][d] buffers and stores them into the bf16
@@ -90,6 +92,9 @@ __global__ void __launch_bounds__(kInsertThreads) kv_stream_insert_kernel(const 
         w.head = st.x + 1 == w.T ? 0 : st.x + 1;
         new_k = st.y + 1 >= p.rebase_every ? 0 : st.y + 1;
         all_rows = new_k == 0;
+    } else if (p.mode == 3) {
+        w.head = st.x;  // already advanced by the kernel that wrote the step's rows
+        all_rows = true;
     } else {
         w.head = st.x;
     }
@@ -107,6 +112,9 @@ __global__ void __launch_bounds__(kInsertThreads) kv_stream_insert_kernel(const 
         if (p.mode == 0) {
             row = ri;
             t = ri;
+        } else if (p.mode == 3) {
+            row = ri;
+            t = -1;
         } else if (p.mode == 1) {
             if (all_rows) {
                 row = ri;
@@ -174,7 +182,7 @@ __global__ void __launch_bounds__(kInsertThreads) kv_stream_insert_kernel(const 
         *reinterpret_cast<uint4*>(ly.V16 + ob) = bf16x8_to_f16x8(vb);
     }
 
-    if (p.mode != 2) {
+    if (p.mode == 0 || p.mode == 1) {
         // Every block read the old state above, before it arrives here; the last
         // block to arrive publishes the new one (the next kernel on the stream
         // starts reading it only after this grid has completed).
@@ -194,7 +202,7 @@ template <int D>
 cudaError_t launch_d(const InsertParams& p, cudaStream_t stream) {
     // Blocks per layer: enough for the rows of an ordinary call (a re-base
     // step loops over the whole window with the same grid).
-    const int rows = p.mode == 0 ? p.w.ring_rows + p.w.X : (p.mode == 1 ? p.w.V * p.w.n + p.w.X : p.N);
+    const int rows = p.mode == 0 || p.mode == 3 ? p.w.ring_rows + p.w.X : (p.mode == 1 ? p.w.V * p.w.n + p.w.X : p.N);
     const long long threads = (long long)rows * p.Hkv * (D / 16);
     const unsigned blocks = unsigned((threads + kInsertThreads - 1) / kInsertThreads);
     return launch_overlapped(kv_stream_insert_kernel<D>, dim3(blocks, unsigned(p.layers)), dim3(kInsertThreads), 0,

@@ -30,10 +30,6 @@ __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
-}
-
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
                  "r"(bytes)
@@ -52,6 +48,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, with acquire semantics at cluster scope: the phase was
+// completed by arrivals of other CTAs of the cluster that released their
+// writes into this CTA's shared memory (mbar_arrive_remote).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: returns false (after setting `code` in *err) once `limit_ns` of
 // wall time has passed without the phase completing. Callers then abandon their
 // loop and head for the kernel's exit path.
@@ -59,19 +70,26 @@ struct BoundedWait {
     unsigned* err;
     uint64_t limit_ns;
     unsigned code;
-    __device__ __forceinline__ bool operator()(uint32_t bar, uint32_t parity) const {
-        if (mbar_try_wait(bar, parity)) return true;
+    template <bool kCluster = false>
+    __device__ __forceinline__ bool try_once(uint32_t bar, uint32_t parity) const {
+        return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+    }
+    // kCluster: acquire at cluster scope (see mbar_try_wait_cluster).
+    template <bool kCluster = false>
+    __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
+        if (try_once<kCluster>(bar, parity)) return true;
         const uint64_t t0 = globaltimer_ns();
         while (true) {
 #pragma unroll 1
             for (int i = 0; i < 32; ++i)
-                if (mbar_try_wait(bar, parity)) return true;
+                if (try_once<kCluster>(bar, parity)) return true;
             if (globaltimer_ns() - t0 > limit_ns) {
                 atomicOr(err, code);
                 return false;
             }
         }
     }
+    __device__ __forceinline__ bool operator()(uint32_t bar, uint32_t parity) const { return wait<false>(bar, parity); }
 };
 
 // ------------------------------------------------- programmatic dependent launch
@@ -107,17 +125,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
-// 3-D tiled bulk tensor store shared -> global (bulk-group completion). Elements
-// outside the tensor's bounds are not written.
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
-    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(src), "r"(x), "r"(y), "r"(z)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until the shared-memory sources of every committed store have been read.
-__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -286,6 +294,21 @@ __device__ __forceinline__ float2 ld_dsmem_f2(uint32_t cluster_addr) {
     return v;
 }
 
+// 16-byte store into another CTA's shared memory (a shared::cluster address
+// from map_to_rank).
+__device__ __forceinline__ void st_dsmem_u4(uint32_t cluster_addr, uint4 v) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Arrive on another CTA's mbarrier (shared::cluster address), releasing this
+// thread's earlier writes at cluster scope: a waiter that observes the phase
+// with mbar_try_wait_cluster sees them.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // Arrive on an mbarrier given by its shared::cluster address (any CTA of the
 // cluster), default (.release.cta) semantics: the data handed over is in TMEM
 // and is ordered by tcgen05.fence::before_thread_sync, so no cluster-scope
@@ -374,16 +397,6 @@ __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
 __device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
 __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -393,10 +406,6 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
-}
-// bf16x2 word -> (lo, hi) as paired fp32 (exact).
-__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
-    return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
 // Packs two floats as bf16x2 (round to nearest even): `lo` in the low 16 bits.

@@ -8,7 +8,8 @@ Every tensor is drawn from numpy's PCG64 seeded with
 ``SeedSequence([workload, layer, step, tensor, call])`` as float32 standard
 normals, multiplied by the workload's scale, then rounded to bf16
 (round-to-nearest-even). Tensor ids: Q = 0, K = 1, V = 2, outlier-row choice = 3;
-the encoder attention's Q, K, V = 10, 11, 12.
+the encoder attention's Q, K, V = 10, 11, 12; the hidden states and the K/V
+projection weight = 20, 21.
 Step 0 is the prefill window (the stream's first call); steps 1.. are window
 steps; ``call`` numbers the verify calls.
 
@@ -23,6 +24,7 @@ import numpy as np
 
 Q_ID, K_ID, V_ID, OUTLIER_ID = 0, 1, 2, 3
 FRAME_Q_ID, FRAME_K_ID, FRAME_V_ID = 10, 11, 12  # encoder attention over the newest frames
+X_ID, W_ID = 20, 21  # hidden states and the stacked K/V projection weight
 
 
 @dataclass(frozen=True)
@@ -155,3 +157,17 @@ def frame_inputs(wid: int, layer: int, step: int, H: int = FRAME_HEADS["H"], Hkv
         K=draw_bf16(wid, layer, step, FRAME_K_ID, 0, (rows, Hkv, d)),
         V=draw_bf16(wid, layer, step, FRAME_V_ID, 0, (rows, Hkv, d)),
     )
+
+
+def hidden_inputs(wid: int, layer: int, step: int, d_model: int) -> np.ndarray:
+    """Hidden states X [tokens(step), d_model] as bf16 bits, ~N(0,1), in the
+    window's token order (as ``window_inputs``)."""
+    wl = WORKLOADS[wid]
+    return draw_bf16(wid, layer, step, X_ID, 0, (wl.tokens(step), d_model))
+
+
+def proj_weight(wid: int, layer: int, d_model: int) -> np.ndarray:
+    """Stacked K/V projection weight W [2*Hkv*d, d_model] as bf16 bits, drawn
+    ~N(0, 1/d_model) so that X W^T is ~N(0, 1) (rows 0 .. Hkv*d-1 give K)."""
+    wl = WORKLOADS[wid]
+    return draw_bf16(wid, layer, 0, W_ID, 0, (2 * wl.Hkv * wl.d, d_model), scale=float(d_model) ** -0.5)
