@@ -624,6 +624,27 @@ def run_ours(args):
             "timing": "CUDA events around the %d calls of a step (one per layer, back to back), per call" % wl.layers,
         }
 
+    # ---- drafted-block verification against the medium window's cache (the
+    # verify workload), replayed from a CUDA graph
+    verify = None
+    vid = 5
+    if rank == 0 and not args.no_wide and vid in WORKLOADS:
+        vs, vblocks = verify_stream(vid, dev)
+        vus = time_verify_graph(vs, vblocks, 8, dev)
+        vs.sync()
+        vs.close()
+        vwl = WORKLOADS[vid]
+        vfl = verify_flops(vwl)
+        verify = {
+            "kernel": "verify_attn",
+            "shape": f"{vwl.verify_tokens}-token drafted blocks after the text of the medium window "
+                     f"(L = {vwl.window_len}, H{vwl.H}/Hkv{vwl.Hkv}/d{vwl.d})",
+            "us_per_call_graph": round(vus, 2),
+            "algorithmic_mflop_per_call": round(vfl / 1e6, 2),
+            "tflops": round(vfl / (vus * 1e-6) / 1e12, 3),
+            "timing": "CUDA events around 8 replays of a graph of 16 calls",
+        }
+
     # ---- end to end through the public C ABI with host buffers
     e2e_steps = max(1, min(args.steps, 5))
     pin = [{x: torch.from_numpy(np.ascontiguousarray(window_inputs(wid, l, 1)[x]).view(np.int16)).pin_memory()
@@ -719,6 +740,7 @@ def run_ours(args):
             "wide_window": wide,
             "frame_encoder": frame,
             "kv_proj": proj,
+            "verify_block": verify,
             "e2e": {
                 "value": round(world * fl_layer * layers / (e2e_ms * 1e-3) / 1e12, 3),
                 "unit": "TFLOP/s",
@@ -741,22 +763,16 @@ def run_ours(args):
     return result
 
 
-def run_verify(args):
-    """Drafted-block verify calls (workload 5): fs_stream_attend_ext of 8-token
-    blocks against the medium window's cache after one step, inputs resident;
-    a "step" is one verify call. The e2e leg copies each block from pinned host
-    memory and the output back inside the timed region."""
+def verify_stream(wid, dev):
+    """A stream holding the verify workload's cache (the medium window after its
+    steps) and device copies of a few drafted blocks."""
     import numpy as np
     import torch
 
-    from streaming_kv_cache_stream_b200.abi import Stream, load
+    from streaming_kv_cache_stream_b200.abi import Stream
     from streaming_kv_cache_stream_b200.inputs import WORKLOADS, verify_inputs, window_inputs
 
-    world, rank, local = dist_setup(args.gpus)
-    load()
-    wid = args.workload
     wl = WORKLOADS[wid]
-    dev = torch.device("cuda", local if world > 1 else 0)
 
     def to_dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -767,8 +783,55 @@ def run_verify(args):
         q = to_dev(inp["Q"])
         s.insert(to_dev(inp["K"]), to_dev(inp["V"]))
         s.attend(q, torch.empty(q.shape, dtype=torch.float32, device=dev))
-    sets = 4
-    blocks = [{x: to_dev(verify_inputs(wid, c)[x]) for x in ("Q", "K", "V")} for c in range(sets)]
+    blocks = [{x: to_dev(verify_inputs(wid, c)[x]) for x in ("Q", "K", "V")} for c in range(4)]
+    return s, blocks
+
+
+def time_verify_graph(s, blocks, replays, dev, calls=16):
+    """fs_stream_attend_ext calls replayed from a CUDA graph of `calls` calls (the
+    pages run the decode loop under CUDA graphs): device microseconds per call."""
+    import torch
+
+    nx, H, d = blocks[0]["Q"].shape
+    gouts = [torch.empty((nx, H, d), dtype=torch.float32, device=dev) for _ in range(2)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for c in range(calls):
+            b = blocks[c % len(blocks)]
+            s.attend_ext(b["Q"], b["K"], b["V"], gouts[c % 2])
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(replays):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    del graph
+    return g0.elapsed_time(g1) * 1e3 / (replays * calls)
+
+
+def run_verify(args):
+    """Drafted-block verify calls (workload 5): fs_stream_attend_ext of 8-token
+    blocks against the medium window's cache after one step, inputs resident;
+    a "step" is one verify call. The e2e leg copies each block from pinned host
+    memory and the output back inside the timed region."""
+    import numpy as np
+    import torch
+
+    from streaming_kv_cache_stream_b200.abi import load
+    from streaming_kv_cache_stream_b200.inputs import WORKLOADS, verify_inputs
+
+    world, rank, local = dist_setup(args.gpus)
+    load()
+    wid = args.workload
+    wl = WORKLOADS[wid]
+    dev = torch.device("cuda", local if world > 1 else 0)
+
+    s, blocks = verify_stream(wid, dev)
+    sets = len(blocks)
     nx = wl.verify_tokens
     out = torch.empty((nx, wl.H, wl.d), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
@@ -813,27 +876,9 @@ def run_verify(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
-    # The same calls replayed from a CUDA graph (the pages run the decode loop
-    # under CUDA graphs): the device time per call without host dispatch.
-    calls = 16
-    gouts = [torch.empty((nx, wl.H, wl.d), dtype=torch.float32, device=dev) for _ in range(2)]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for c in range(calls):
-            b = blocks[c % sets]
-            s.attend_ext(b["Q"], b["K"], b["V"], gouts[c % 2])
-    for _ in range(3):
-        graph.replay()
-    torch.cuda.synchronize()
-    replays = max(1, args.steps // calls)
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record(stream)
-    for _ in range(replays):
-        graph.replay()
-    g1.record(stream)
-    torch.cuda.synchronize()
-    graph_ms = max_over_ranks(g0.elapsed_time(g1), world) / (replays * calls)
-    del graph
+    # The same calls replayed from a CUDA graph: the device time per call
+    # without host dispatch.
+    graph_ms = max_over_ranks(time_verify_graph(s, blocks, max(1, args.steps // 16), dev) / 1e3, world)
     s.sync()
     s.close()
     if world > 1:
