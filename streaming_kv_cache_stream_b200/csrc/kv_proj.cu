@@ -15,17 +15,18 @@
 //
 // Work split: a cluster of two CTAs owns a 128 x 256 tile of X W^T (128
 // tokens, 256 output columns) and splits d_model between them (split-K): each
-// CTA streams its half of the 64-column blocks of X and W through a 4-stage
+// CTA streams its half of the 64-column blocks of X and W through a 3-stage
 // TMA ring (128-byte swizzle) and one thread issues bf16 tcgen05 MMAs of
 // M = 128, N = 256 (the shape that keeps the tensor pipe busiest on one SM)
 // into an fp32 accumulator in TMEM. Then each CTA stores the partial sums of
 // the peer's 128 columns into a receive buffer in the peer's shared memory
 // (distributed shared memory, signalled through the peer's mbarrier), adds the
-// peer's partial to its own 128 columns, and finishes them. Thread (g, r) of the two warpgroups holds token
-// m0 + r and 64 of the columns, chosen so that the rotate-half partners
-// (i, i + d/2) of a key are in the same thread. Results are staged in shared
-// memory and written out as whole contiguous cache rows. The last CTA to
-// finish advances the ring state (head, k) as kv_stream_insert does.
+// peer's partial to its own 128 columns, and finishes them. Thread (g, r) of
+// the two warpgroups holds token m0 + r and 64 of the columns, chosen so that
+// the rotate-half partners (i, i + d/2) of a key are in the same thread.
+// Results are staged in shared memory and written out as whole contiguous
+// cache rows. The last CTA to finish advances the ring state (head, k) as
+// kv_stream_insert does.
 #include "fs_internal.cuh"
 #include "sm100.cuh"
 
@@ -96,8 +97,10 @@ __device__ __forceinline__ bool stage_pairs(const float (&ya)[32], const float (
     const int ca = a0 / 8, cb = (a0 + D / 2) / 8;  // first 16-byte chunk of each part
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        *reinterpret_cast<uint4*>(out + stage_off<D>(r, ca + c)) = make_uint4(ba[4 * c], ba[4 * c + 1], ba[4 * c + 2], ba[4 * c + 3]);
-        *reinterpret_cast<uint4*>(out + stage_off<D>(r, cb + c)) = make_uint4(bb[4 * c], bb[4 * c + 1], bb[4 * c + 2], bb[4 * c + 3]);
+        *reinterpret_cast<uint4*>(out + stage_off<D>(r, ca + c)) =
+            make_uint4(ba[4 * c], ba[4 * c + 1], ba[4 * c + 2], ba[4 * c + 3]);
+        *reinterpret_cast<uint4*>(out + stage_off<D>(r, cb + c)) =
+            make_uint4(bb[4 * c], bb[4 * c + 1], bb[4 * c + 2], bb[4 * c + 3]);
     }
     if (!operands) return true;
     bool in_range = true;
