@@ -62,6 +62,16 @@ def verify_flops(wl):
     return 4.0 * wl.d * wl.H * sum(wl.window_len + t + 1 for t in range(wl.verify_tokens))
 
 
+def frame_flops(wl, heads=None):
+    """Algorithmic FLOPs of one encoder-attention call over the newest frame of
+    every view: each of a view's n tokens sees all n (QK^T and PV, 2 each per
+    element), 4 d H n^2 per view."""
+    from streaming_kv_cache_stream_b200.inputs import FRAME_HEADS
+
+    h = heads or FRAME_HEADS
+    return 4.0 * h["d"] * h["H"] * wl.views * wl.tok_per_frame ** 2
+
+
 def insert_algorithmic_bytes(wl):
     """Bytes one layer's window-step insert must move: read the step's K and V
     (bf16) and write them into the ring, i.e. 2 tensors x (read + write) x
@@ -382,7 +392,7 @@ def time_frame_attention(wid, calls, dev):
     import torch
 
     from streaming_kv_cache_stream_b200.abi import Stream
-    from streaming_kv_cache_stream_b200.inputs import FRAME_HEADS, WORKLOADS, frame_inputs
+    from streaming_kv_cache_stream_b200.inputs import WORKLOADS, frame_inputs
 
     wl = WORKLOADS[wid]
 
@@ -416,8 +426,7 @@ def time_frame_attention(wid, calls, dev):
     s.sync()
     s.close()
     us = [a.elapsed_time(c) * 1e3 / 10 for a, c in ev]
-    flops = 4.0 * FRAME_HEADS["d"] * FRAME_HEADS["H"] * wl.views * wl.tok_per_frame ** 2
-    return us, flops
+    return us, frame_flops(wl)
 
 
 def time_kv_proj(wid, steps, warmup, dev):

@@ -65,3 +65,32 @@ def test_verify_flops_match_the_golden_pair_count():
         golden = json.load(f)
     wl = WORKLOADS[5]
     assert bench.verify_flops(wl) == pytest.approx(4.0 * wl.d * wl.H * golden["2"]["verify_pairs"])
+
+
+def test_insert_bytes_follow_the_definition():
+    """Algorithmic insert bytes per layer step: read the step's K and V and
+    write them into the ring, 4 N_new Hkv d bytes of bf16 (7,995,392 at the
+    driving shape); the kernel's own traffic adds the fp16 operand rows."""
+    import bench
+    from streaming_kv_cache_stream_b200.inputs import WORKLOADS
+
+    wl = WORKLOADS[3]
+    assert bench.insert_algorithmic_bytes(wl) == 4 * wl.step_tokens * wl.Hkv * wl.d * 2 == 7995392
+    impl = bench.insert_implementation_bytes(wl)
+    assert impl >= 1.75 * bench.insert_algorithmic_bytes(wl)
+
+
+def test_frame_flops_count_the_frame_pairs():
+    """Encoder attention: every token of a view's frame sees the whole frame,
+    so a call does 4 d H n^2 per view; checked against a brute-force count of
+    the (query, key) pairs of the oracle's per-view mask."""
+    import numpy as np
+
+    import bench
+    from streaming_kv_cache_stream_b200.inputs import Workload
+
+    wl = Workload("f", 3, 2, 5, 0, H=4, Hkv=2, d=8)
+    heads = dict(H=4, Hkv=2, d=8)
+    view = np.repeat(np.arange(wl.views), wl.tok_per_frame)
+    pairs = int((view[:, None] == view[None, :]).sum())
+    assert bench.frame_flops(wl, heads) == 4.0 * heads["d"] * heads["H"] * pairs
