@@ -73,3 +73,7 @@ def test_null_handle_calls_fail_cleanly(lib):
     assert lib.fs_stream_append(None, None, None, 1) == abi.FS_ERR_ARG
     assert lib.fs_stream_insert_batch(None, 1, None, None) == abi.FS_ERR_ARG
     assert lib.fs_stream_insert_batch(None, 0, None, None) == abi.FS_ERR_ARG
+    assert lib.fs_stream_insert_proj(None, None, None, 4096) == abi.FS_ERR_ARG
+    assert lib.fs_frame_attend(None, None, None, None, 16, 16, 64, None) == abi.FS_ERR_ARG
+    assert lib.fs_stream_attend_ext_static(None, None, None, None, 8, None) == abi.FS_ERR_ARG
+    assert lib.fs_stream_step_host(None, None, None, None, None) == abi.FS_ERR_ARG
